@@ -1,0 +1,206 @@
+/*
+ * nvfp4decode.h -- C ABI of libnvfp4decode.so, the NVFP4 weight-streaming
+ * decode round for NVIDIA B200 (sm_100a).
+ *
+ * The operation (ignis README, section "The decode round"; "Why ignis", tile
+ * "One round for every lane"): up to eight decode lanes share one pass over
+ * the weights,
+ *
+ *     Y[M][N] = X[M][K] . dequant(W)^T,        M = 1..8,
+ *     dequant(W)[n][k] = gscale * e2m1(q[n][k]) * e4m3(s[n][k/16]),
+ *
+ * with W stored as NVFP4: 4-bit E2M1 elements and one E4M3 scale per 16
+ * consecutive K values ("Models and artifacts", section "The artifact"),
+ * plus one FP32 global scale.  X is BF16, accumulation is FP32.  The whole
+ * round is replayed from one CUDA graph per batch width (README, "The decode
+ * round"); the step-level boundary is flat and device-resident (README,
+ * introduction: "flat, device-resident step-level C ABI").
+ *
+ * Conventions shared by every call:
+ *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *    owns every buffer; the library never frees caller memory.
+ *  - Device pointers must be 16-byte aligned (else NVFP4_ERR_ALIGN).
+ *  - M in 1..8 (else NVFP4_ERR_M); N >= 1; K >= 16 and K % 16 == 0
+ *    (else NVFP4_ERR_SHAPE).
+ *  - X, Y and H are dense row-major with leading dimension K, N and N.
+ *  - Calls never throw, abort or trap.  Asynchronous calls return once the
+ *    work is enqueued on `stream`; a device fault surfaces at the caller's
+ *    next synchronisation, or as NVFP4_ERR_CUDA here with the CUDA error code
+ *    kept for nvfp4_last_cuda_error().
+ *  - `stream` may be NULL (the legacy default stream).
+ */
+#ifndef NVFP4DECODE_H
+#define NVFP4DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* the same handle as cudaStream_t */
+typedef struct nvfp4_round nvfp4_round;     /* opaque graph-replay handle */
+
+enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_ARG = -1,       /* NULL pointer, bad kind, bad count */
+    NVFP4_ERR_M = -2,         /* M outside 1..8 */
+    NVFP4_ERR_SHAPE = -3,     /* N < 1, K < 16 or K % 16 != 0, size overflow */
+    NVFP4_ERR_ALIGN = -4,     /* a device pointer is not 16-byte aligned */
+    NVFP4_ERR_BAD_SCALE = -5, /* a scale byte is an E4M3 NaN code (0x7F / 0xFF) */
+    NVFP4_ERR_CUDA = -6,      /* a CUDA runtime call failed; see nvfp4_last_cuda_error() */
+    NVFP4_ERR_CAPTURE = -7,   /* first use of a device while its stream is being captured */
+    NVFP4_ERR_DEVICE = -8     /* a kernel's bounded wait gave up; see nvfp4_device_status() */
+};
+
+/*
+ * Sizes of the device-layout planes of an N x K NVFP4 matrix.
+ *
+ * The device layout ("Models and artifacts", "The artifact": the kernels read
+ * the weight planes directly) keeps the canonical byte counts per element --
+ * half a byte per weight and one scale byte per 16 -- but permutes them into
+ * 32-row x 64-column units (1024 nibble bytes + 128 scale bytes each) so that
+ * every warp streams one contiguous run of bytes.  N is padded to a multiple
+ * of 32 and K to a multiple of 64 with zero codes and zero scales.
+ * Writes *wq_bytes and *ws_bytes (host pointers).  Pure host call.
+ */
+int nvfp4_packed_bytes(int64_t N, int64_t K, size_t* wq_bytes, size_t* ws_bytes);
+
+/*
+ * Load-time pack: canonical planes -> device layout, plus a scan for NaN
+ * scale codes.  Canonical planes ("Models and artifacts", "The artifact"):
+ *   wq_canon  u8[N][K/2]: element k of row n in byte k/2, the even element
+ *             in the low nibble and the odd element in the high nibble;
+ *   ws_canon  u8[N][K/16]: E4M3 scale of k in [16b, 16b+15] of row n.
+ * wq_dev / ws_dev receive nvfp4_packed_bytes() bytes each.  The call
+ * synchronises `stream` and returns NVFP4_ERR_BAD_SCALE if any scale byte is
+ * 0x7F or 0xFF (the planes are still written).  Not reentrant across host
+ * threads on one device (serialised internally).
+ */
+int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N, int64_t K,
+                     uint8_t* wq_dev, uint8_t* ws_dev, nvfp4_stream_t stream);
+
+/*
+ * The decode GEMM, asynchronous:  Y[m][n] = gscale * sum_k X[m][k] w[n][k].
+ *   X   bf16 [M][K];  Y float [M][N];  wq_dev / ws_dev from nvfp4_pack_check.
+ * The weights are read once per call for all M lanes (README, "The decode
+ * round").  Split-K partial sums are combined in a fixed order, so results
+ * are bit-identical from call to call.  Uses a per-device workspace that the
+ * first call on a device allocates; that first call must not be made while
+ * `stream` is being captured (NVFP4_ERR_CAPTURE).  Calls on one device that
+ * overlap in time share that workspace and must not run concurrently.
+ */
+int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
+                      float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);
+
+/*
+ * Fused MLP front half, asynchronous, one launch for both projections:
+ *   g = gscale_gate * X . Wg^T,  u = gscale_up * X . Wu^T,
+ *   H[m][n] = bf16( silu(g) * u ),  silu(g) = g / (1 + exp(-g)).
+ * X bf16 [M][K]; H bf16 [M][Nff]; the gate and up matrices are separate
+ * Nff x K matrices in device layout.  Same workspace rules as
+ * nvfp4_gemm_decode.
+ */
+int nvfp4_gemm_gateup_silu(const void* X, int M,
+                           const uint8_t* wq_gate, const uint8_t* ws_gate, float gscale_gate,
+                           const uint8_t* wq_up, const uint8_t* ws_up, float gscale_up,
+                           void* H, int64_t Nff, int64_t K, nvfp4_stream_t stream);
+
+/* One node of a decode round. */
+enum { NVFP4_DESC_GEMM = 0, NVFP4_DESC_GATEUP_SILU = 1 };
+typedef struct {
+    int kind;              /* NVFP4_DESC_GEMM or NVFP4_DESC_GATEUP_SILU */
+    const void* X;         /* bf16 [M][K], rows for M = 8 must be allocated */
+    const uint8_t* wq;     /* device-layout planes (gate for GATEUP_SILU) */
+    const uint8_t* ws;
+    float gscale;
+    const uint8_t* wq2;    /* up projection planes (GATEUP_SILU only, else NULL) */
+    const uint8_t* ws2;
+    float gscale2;
+    void* out;             /* float [M][N] (GEMM) or bf16 [M][N] (GATEUP_SILU) */
+    int64_t N, K;
+} nvfp4_gemm_desc;
+
+/*
+ * Build a decode round: the n descriptors are launched in order, each as a
+ * programmatic-dependent launch of the previous one (a PDL chain: every node
+ * prefetches its weights before waiting on its predecessor), and captured
+ * once per batch width M = 1..8 into eight CUDA graphs (README, "The decode
+ * round": per-width CUDA graphs, widths 1..8).  The descriptor array is
+ * copied; the buffers it names must outlive the round.  Allocates the graphs
+ * and the per-device workspace.  Synchronous; *out is a host pointer.
+ */
+int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_round** out);
+
+/* Number of kernel nodes in each of the round's graphs (host call). */
+int nvfp4_round_nodes(const nvfp4_round* r, int* nodes);
+
+/*
+ * Replay the width-M graph on `stream` (one graph launch, asynchronous).
+ * The graph reads whatever the descriptor buffers hold when it runs.
+ * A round handle is not thread-safe.
+ */
+int nvfp4_round_replay(nvfp4_round* r, int M, nvfp4_stream_t stream);
+
+/*
+ * The same replay with host buffers at both ends, all on `stream`:
+ * copy x_bytes from x_host (host) to x_dev, replay the width-M graph, copy
+ * y_bytes from y_dev to y_host (host).  Asynchronous; pinned host memory
+ * makes the copies asynchronous too.
+ */
+int nvfp4_round_replay_host(nvfp4_round* r, int M, const void* x_host, void* x_dev,
+                            size_t x_bytes, const void* y_dev, void* y_host, size_t y_bytes,
+                            nvfp4_stream_t stream);
+
+/* Release the graphs of a round (synchronises nothing; NULL is accepted). */
+int nvfp4_round_destroy(nvfp4_round* r);
+
+/*
+ * Test aid: the dequantised weights exactly as the GEMM kernels form them,
+ * W[n][k] = fp32(e2m1 * e4m3 * gscale), float [N][K] (unpadded).  Asynchronous.
+ */
+int nvfp4_dequant_debug(const uint8_t* wq_dev, const uint8_t* ws_dev, float gscale, float* W,
+                        int64_t N, int64_t K, nvfp4_stream_t stream);
+
+/*
+ * Test aid: device layout -> canonical planes (the inverse of the pack).
+ * wq_canon u8[N][K/2], ws_canon u8[N][K/16].  Asynchronous.
+ */
+int nvfp4_unpack_debug(const uint8_t* wq_dev, const uint8_t* ws_dev, int64_t N, int64_t K,
+                       uint8_t* wq_canon, uint8_t* ws_canon, nvfp4_stream_t stream);
+
+/*
+ * Host-side model of the device layout, for CPU tests (no GPU needed):
+ * dequantise one packed 32 x 64 unit with the same bit placement and the
+ * same bf16 arithmetic the kernels use.  q_unit: 1024 host bytes, s_unit:
+ * 128 host bytes; W: float [32][64] host output (gscale applied).
+ */
+int nvfp4_host_dequant_unit(const uint8_t* q_unit, const uint8_t* s_unit, float gscale,
+                            float* W);
+
+/* Host-side pack of one unit: canonical host planes -> one 1024 + 128 byte unit. */
+int nvfp4_host_pack_unit(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N, int64_t K,
+                         int64_t tile, int64_t chunk, uint8_t* q_unit, uint8_t* s_unit);
+
+/* Text for a status code (static storage). */
+const char* nvfp4_status_string(int status);
+
+/* CUDA error code of the last NVFP4_ERR_CUDA on this host thread (0 if none). */
+int nvfp4_last_cuda_error(void);
+
+/*
+ * Device-side status of the current device: 0 when every kernel finished its
+ * bounded waits, else a nonzero code.  Reading it synchronises the device;
+ * a nonzero status also clears the flag and re-zeroes the split-K counters.
+ */
+int nvfp4_device_status(void);
+
+/* Library version, e.g. 100 for 1.0. */
+int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4DECODE_H */
