@@ -1,0 +1,477 @@
+#!/usr/bin/env python3
+"""Benchmark of the NVFP4 weight-streaming decode round on B200.
+
+One step = one replay of the full synthetic decode round (64 layers of
+q/k/v, o, fused gate/up + SiLU-multiply and down GEMMs, plus the vocabulary
+head; about 13.84 GB of NVFP4 weights) at batch width M (default 8), from
+its per-width CUDA graph.  The metric is the HBM weight-stream rate in GB/s
+(algorithmic weight bytes per round / round time) with the round time in ms
+alongside; a per-M sweep of single GEMMs is reported as detail.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--width M] [--impl reference]
+
+For N > 1 it runs under torchrun, one independent replica per GPU (the round
+does not shard: replicas only), timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 decode GEMM HBM GB/s and % of B200 peak at M=1..8; full round ms"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["gemm.cu", "dequant.cuh", "layout.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--width", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "nvfp4_weight_streaming_decode_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per round from the committed ncu summary, if its kernel hash is current."""
+    path = os.path.join(ROOT, "profiles", "decode_gemm_round_m8_traffic.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_hash") != kernel_hash():
+            return None
+        return float(kv["dram_bytes_per_round"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+
+def oracle_sample(device, seconds_budget):
+    """Time the float64 oracle on a bounded row sample of layer 0's q/k/v GEMM
+    (K = 5120, M = 8); returns (GB/s of weights processed, cores, description)."""
+    import numpy as np
+
+    import oracle
+    from nvfp4_weight_streaming_decode_b200 import synth
+    hidden = synth.WORKLOADS[4]["hidden"]
+    q_full, s_full = synth.torch_matrix(4, 0, 3 * hidden, hidden, device)
+    X = synth.torch_activations(4, 0, 8, hidden, device)
+    Xb = X.view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+    rows_total = 0
+    elapsed = 0.0
+    r = 16
+    while True:
+        rows = min(r, q_full.shape[0])
+        q = q_full[:rows].cpu().numpy()
+        s = s_full[:rows].cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.gemm(Xb, q, s, synth.GSCALE)
+        dt = time.perf_counter() - t0
+        rows_total += rows
+        elapsed += dt
+        if elapsed >= seconds_budget or rows == q_full.shape[0]:
+            break
+        r = int(min(q_full.shape[0], max(2 * r, r * (seconds_budget - elapsed) / max(dt, 1e-3) * 0.5)))
+    gbs = rows_total * hidden * (0.5 + 1 / 16) / elapsed / 1e9
+    return gbs, oracle.threads(), f"oracle GEMM, M=8, {rows_total} rows of layer-0 q/k/v (K={hidden}) in {elapsed:.1f} s"
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    from nvfp4_weight_streaming_decode_b200 import synth
+    hidden = synth.WORKLOADS[4]["hidden"]
+    q_full, s_full = synth.matrix(4, 0, 3 * hidden, hidden)
+    Xb = synth.activations(synth.rng(4, 0), args.width, hidden)
+    per_step_rows = 128
+    times = []
+    rows_done = 0
+    for i in range(args.warmup + args.steps):
+        lo = (i * per_step_rows) % (q_full.shape[0] - per_step_rows)
+        q = np.ascontiguousarray(q_full[lo:lo + per_step_rows])
+        s = np.ascontiguousarray(s_full[lo:lo + per_step_rows])
+        t0 = time.perf_counter()
+        oracle.gemm(Xb, q, s, synth.GSCALE)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            rows_done += per_step_rows
+    total = sum(times)
+    gbs = rows_done * hidden * (0.5 + 1 / 16) / total / 1e9
+    sample = (f"float64 oracle GEMM, M={args.width}, {per_step_rows} rows of the round's layer-0 "
+              f"q/k/v matrix (K={hidden}) per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / max(1, len(times)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "round_64layers_head_m1to8 (sampled rows, CPU oracle)",
+                   "width_M": args.width, "hidden": hidden},
+        "cpu_baseline": {"value": gbs, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU legs
+
+def gemm_sweep(dev, hbm_peak):
+    """Standalone decode GEMMs per workload and width; CUDA events over
+    back-to-back launches with enough rotating weight copies to exceed L2."""
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi, synth
+    from nvfp4_weight_streaming_decode_b200.workloads import BYTES_PER_WEIGHT, make_matrix
+    out = []
+    stream = torch.cuda.current_stream()
+
+    def time_calls(fn, n_iter, copies):
+        for i in range(3):
+            fn(i % copies)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n_iter):
+            fn(i % copies)
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / n_iter * 1e-3
+
+    # single projection N = K = 5120, 16 copies (236 MB > L2)
+    mats = [make_matrix(1, 500 + c, 5120, 5120, dev) for c in range(16)]
+    for M in range(1, 9):
+        X = synth.torch_activations(1, M, M, 5120, dev)
+        Y = torch.empty((M, 5120), dtype=torch.float32, device=dev)
+
+        def f(c, M=M, X=X, Y=Y):
+            m = mats[c]
+            abi.check(abi.nvfp4_gemm_decode(X.data_ptr(), M, m.wq.data_ptr(), m.ws.data_ptr(), synth.GSCALE,
+                                            Y.data_ptr(), 5120, 5120, stream.cuda_stream))
+        t = time_calls(f, 200, len(mats))
+        b = 5120 * 5120 * BYTES_PER_WEIGHT + 2 * M * 5120 + 4 * M * 5120
+        out.append({"workload": "proj_n5120_k5120", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
+                    "frac": b / t / 1e9 / hbm_peak})
+    del mats
+    # head N = 151936, K = 5120 (438 MB > L2)
+    head = make_matrix(3, 0, 151936, 5120, dev, synth.EXP_LOGU_M6_4)
+    for M in (1, 4, 8):
+        X = synth.torch_activations(3, M, M, 5120, dev)
+        Y = torch.empty((M, 151936), dtype=torch.float32, device=dev)
+
+        def f(c, M=M, X=X, Y=Y):
+            abi.check(abi.nvfp4_gemm_decode(X.data_ptr(), M, head.wq.data_ptr(), head.ws.data_ptr(),
+                                            synth.GSCALE, Y.data_ptr(), 151936, 5120, stream.cuda_stream))
+        t = time_calls(f, 30, 1)
+        b = 151936 * 5120 * BYTES_PER_WEIGHT + 2 * M * 5120 + 4 * M * 151936
+        out.append({"workload": "head_n151936_k5120", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
+                    "frac": b / t / 1e9 / hbm_peak})
+    del head
+    # fused MLP: gate/up 2 x 17408 x 5120 then down 5120 x 17408, 2 copies (300 MB > L2)
+    sets = [(make_matrix(2, 600 + 3 * c, 17408, 5120, dev), make_matrix(2, 601 + 3 * c, 17408, 5120, dev),
+             make_matrix(2, 602 + 3 * c, 5120, 17408, dev)) for c in range(2)]
+    for M in (1, 8):
+        X = synth.torch_activations(2, M, M, 5120, dev)
+        H = torch.empty((M, 17408), dtype=torch.bfloat16, device=dev)
+        Y = torch.empty((M, 5120), dtype=torch.float32, device=dev)
+
+        def fg(c, M=M, X=X, H=H):
+            g, u, _ = sets[c]
+            abi.check(abi.nvfp4_gemm_gateup_silu(X.data_ptr(), M, g.wq.data_ptr(), g.ws.data_ptr(), synth.GSCALE,
+                                                 u.wq.data_ptr(), u.ws.data_ptr(), synth.GSCALE, H.data_ptr(),
+                                                 17408, 5120, stream.cuda_stream))
+
+        def fd(c, M=M, H=H, Y=Y):
+            d = sets[c][2]
+            abi.check(abi.nvfp4_gemm_decode(H.data_ptr(), M, d.wq.data_ptr(), d.ws.data_ptr(), synth.GSCALE,
+                                            Y.data_ptr(), 5120, 17408, stream.cuda_stream))
+        t = time_calls(fg, 60, 2)
+        b = 2 * 17408 * 5120 * BYTES_PER_WEIGHT + 2 * M * 5120 + 2 * M * 17408
+        out.append({"workload": "mlp_gateup_2x17408_k5120", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
+                    "frac": b / t / 1e9 / hbm_peak})
+        t = time_calls(fd, 60, 2)
+        b = 5120 * 17408 * BYTES_PER_WEIGHT + 2 * M * 17408 + 4 * M * 5120
+        out.append({"workload": "mlp_down_n5120_k17408", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
+                    "frac": b / t / 1e9 / hbm_peak})
+    del sets
+    torch.cuda.synchronize()
+    return out
+
+
+def round_io_bytes(r, M):
+    """Algorithmic activation bytes of one round: X read and outputs written, per node."""
+    from nvfp4_weight_streaming_decode_b200 import abi
+    total = 0
+    for (_, kind, _, _, mkeys) in r.nodes:
+        m0 = r.mats[mkeys[0]]
+        total += 2 * M * m0.K + (4 if kind == abi.NVFP4_DESC_GEMM else 2) * M * m0.N
+    return total
+
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from nvfp4_weight_streaming_decode_b200 import abi, build, synth
+    from nvfp4_weight_streaming_decode_b200.workloads import SyntheticRound
+    build.build()
+    abi.load()
+    hbm_peak, peak_kind = peaks()
+    M = args.width
+    w = synth.WORKLOADS[4]
+
+    r = SyntheticRound.build(dev, layers=args.layers, hidden=w["hidden"], ffn=w["ffn"], vocab=w["vocab"])
+    rnd = abi.Round(r.descs)
+    nodes = rnd.nodes
+    weight_bytes = r.weight_bytes
+    io_bytes = round_io_bytes(r, M)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            rnd.replay(M, stream)
+    torch.cuda.synchronize()
+
+    # per-width round times (detail): 20 replays each
+    by_width = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for m in range(1, 9):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                rnd.replay(m, stream)
+            e0.record(stream)
+            for _ in range(20):
+                rnd.replay(m, stream)
+            e1.record(stream)
+        e1.synchronize()
+        by_width[m] = e0.elapsed_time(e1) / 20
+
+    # the timed region: K replays at width M
+    clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            rnd.replay(M, stream)
+        e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    elapsed_s = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world)
+    ms_per_step = elapsed_s * 1e3 / args.steps
+    value = world * weight_bytes * args.steps / elapsed_s / 1e9
+
+    # end to end through the C ABI with host buffers: H2D of the layer-0 input,
+    # the replay, D2H of the logits, every step
+    x_host = torch.empty((M, w["hidden"]), dtype=torch.bfloat16).pin_memory()
+    x_host.copy_(r.bufs["x0"][:M].cpu())
+    y_host = torch.empty((M, w["vocab"]), dtype=torch.float32).pin_memory()
+    e2e_steps = max(10, args.steps // 4)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            rnd.replay_host(M, x_host, r.bufs["x0"], r.bufs["logits"][:M], y_host, stream)
+        barrier(world)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            rnd.replay_host(M, x_host, r.bufs["x0"], r.bufs["logits"][:M], y_host, stream)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world)
+    e2e_value = world * weight_bytes * e2e_steps / e2e_s / 1e9
+
+    # roofline of the decode GEMM kernel over the round: every node is a launch of it
+    per_launch_bytes = (weight_bytes + io_bytes) / nodes
+    per_launch_s = (elapsed_s / args.steps) / nodes
+    achieved = per_launch_bytes / per_launch_s / 1e9
+    traffic_round = profiled_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak,
+                "traffic": (traffic_round / nodes) if traffic_round else None,
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "kernel": "decode_gemm_kernel (all round nodes)"}
+
+    sweep = None
+    if rank == 0 and not args.no_sweep:
+        del rnd
+        sweep = gemm_sweep(dev, hbm_peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, cores, sample = oracle_sample(dev, 12.0)
+        cpu = {"value": gbs, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random NVFP4 codes/scales, N(0,1) bf16 activations)",
+            "config": {"workload": "round_64layers_head_m1to8", "width_M": M, "layers": args.layers,
+                       "hidden": w["hidden"], "ffn": w["ffn"], "vocab": w["vocab"],
+                       "weight_bytes_per_round": weight_bytes, "graph_nodes": nodes,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (13.8 GB of weights per round)"},
+            "round_ms": ms_per_step,
+            "round_ms_by_width": by_width,
+            "round_GBps_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 for m, t in by_width.items()},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_host.numel() * 2,
+                    "d2h_bytes_per_step": y_host.numel() * 4, "ms_per_step": e2e_s * 1e3 / e2e_steps},
+            "gpu_launches": nodes * args.steps,
+            "clocks": clk,
+            "gemm_sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -35,6 +35,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -65,7 +71,7 @@ enum {
  * of 32 and K to a multiple of 64 with zero codes and zero scales.
  * Writes *wq_bytes and *ws_bytes (host pointers).  Pure host call.
  */
-int nvfp4_packed_bytes(int64_t N, int64_t K, size_t* wq_bytes, size_t* ws_bytes);
+NVFP4_API int nvfp4_packed_bytes(int64_t N, int64_t K, size_t* wq_bytes, size_t* ws_bytes);
 
 /*
  * Load-time pack: canonical planes -> device layout, plus a scan for NaN
@@ -78,7 +84,7 @@ int nvfp4_packed_bytes(int64_t N, int64_t K, size_t* wq_bytes, size_t* ws_bytes)
  * 0x7F or 0xFF (the planes are still written).  Not reentrant across host
  * threads on one device (serialised internally).
  */
-int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N, int64_t K,
+NVFP4_API int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N, int64_t K,
                      uint8_t* wq_dev, uint8_t* ws_dev, nvfp4_stream_t stream);
 
 /*
@@ -91,7 +97,7 @@ int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N
  * `stream` is being captured (NVFP4_ERR_CAPTURE).  Calls on one device that
  * overlap in time share that workspace and must not run concurrently.
  */
-int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
+NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                       float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);
 
 /*
@@ -102,7 +108,7 @@ int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t
  * Nff x K matrices in device layout.  Same workspace rules as
  * nvfp4_gemm_decode.
  */
-int nvfp4_gemm_gateup_silu(const void* X, int M,
+NVFP4_API int nvfp4_gemm_gateup_silu(const void* X, int M,
                            const uint8_t* wq_gate, const uint8_t* ws_gate, float gscale_gate,
                            const uint8_t* wq_up, const uint8_t* ws_up, float gscale_up,
                            void* H, int64_t Nff, int64_t K, nvfp4_stream_t stream);
@@ -131,17 +137,17 @@ typedef struct {
  * copied; the buffers it names must outlive the round.  Allocates the graphs
  * and the per-device workspace.  Synchronous; *out is a host pointer.
  */
-int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_round** out);
+NVFP4_API int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_round** out);
 
 /* Number of kernel nodes in each of the round's graphs (host call). */
-int nvfp4_round_nodes(const nvfp4_round* r, int* nodes);
+NVFP4_API int nvfp4_round_nodes(const nvfp4_round* r, int* nodes);
 
 /*
  * Replay the width-M graph on `stream` (one graph launch, asynchronous).
  * The graph reads whatever the descriptor buffers hold when it runs.
  * A round handle is not thread-safe.
  */
-int nvfp4_round_replay(nvfp4_round* r, int M, nvfp4_stream_t stream);
+NVFP4_API int nvfp4_round_replay(nvfp4_round* r, int M, nvfp4_stream_t stream);
 
 /*
  * The same replay with host buffers at both ends, all on `stream`:
@@ -149,25 +155,25 @@ int nvfp4_round_replay(nvfp4_round* r, int M, nvfp4_stream_t stream);
  * y_bytes from y_dev to y_host (host).  Asynchronous; pinned host memory
  * makes the copies asynchronous too.
  */
-int nvfp4_round_replay_host(nvfp4_round* r, int M, const void* x_host, void* x_dev,
+NVFP4_API int nvfp4_round_replay_host(nvfp4_round* r, int M, const void* x_host, void* x_dev,
                             size_t x_bytes, const void* y_dev, void* y_host, size_t y_bytes,
                             nvfp4_stream_t stream);
 
 /* Release the graphs of a round (synchronises nothing; NULL is accepted). */
-int nvfp4_round_destroy(nvfp4_round* r);
+NVFP4_API int nvfp4_round_destroy(nvfp4_round* r);
 
 /*
  * Test aid: the dequantised weights exactly as the GEMM kernels form them,
  * W[n][k] = fp32(e2m1 * e4m3 * gscale), float [N][K] (unpadded).  Asynchronous.
  */
-int nvfp4_dequant_debug(const uint8_t* wq_dev, const uint8_t* ws_dev, float gscale, float* W,
+NVFP4_API int nvfp4_dequant_debug(const uint8_t* wq_dev, const uint8_t* ws_dev, float gscale, float* W,
                         int64_t N, int64_t K, nvfp4_stream_t stream);
 
 /*
  * Test aid: device layout -> canonical planes (the inverse of the pack).
  * wq_canon u8[N][K/2], ws_canon u8[N][K/16].  Asynchronous.
  */
-int nvfp4_unpack_debug(const uint8_t* wq_dev, const uint8_t* ws_dev, int64_t N, int64_t K,
+NVFP4_API int nvfp4_unpack_debug(const uint8_t* wq_dev, const uint8_t* ws_dev, int64_t N, int64_t K,
                        uint8_t* wq_canon, uint8_t* ws_canon, nvfp4_stream_t stream);
 
 /*
@@ -176,28 +182,28 @@ int nvfp4_unpack_debug(const uint8_t* wq_dev, const uint8_t* ws_dev, int64_t N, 
  * same bf16 arithmetic the kernels use.  q_unit: 1024 host bytes, s_unit:
  * 128 host bytes; W: float [32][64] host output (gscale applied).
  */
-int nvfp4_host_dequant_unit(const uint8_t* q_unit, const uint8_t* s_unit, float gscale,
+NVFP4_API int nvfp4_host_dequant_unit(const uint8_t* q_unit, const uint8_t* s_unit, float gscale,
                             float* W);
 
 /* Host-side pack of one unit: canonical host planes -> one 1024 + 128 byte unit. */
-int nvfp4_host_pack_unit(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N, int64_t K,
+NVFP4_API int nvfp4_host_pack_unit(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N, int64_t K,
                          int64_t tile, int64_t chunk, uint8_t* q_unit, uint8_t* s_unit);
 
 /* Text for a status code (static storage). */
-const char* nvfp4_status_string(int status);
+NVFP4_API const char* nvfp4_status_string(int status);
 
 /* CUDA error code of the last NVFP4_ERR_CUDA on this host thread (0 if none). */
-int nvfp4_last_cuda_error(void);
+NVFP4_API int nvfp4_last_cuda_error(void);
 
 /*
  * Device-side status of the current device: 0 when every kernel finished its
  * bounded waits, else a nonzero code.  Reading it synchronises the device;
  * a nonzero status also clears the flag and re-zeroes the split-K counters.
  */
-int nvfp4_device_status(void);
+NVFP4_API int nvfp4_device_status(void);
 
 /* Library version, e.g. 100 for 1.0. */
-int nvfp4_version(void);
+NVFP4_API int nvfp4_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,303 @@
+"""ctypes binding of libnvfp4decode.so -- argument marshalling only.
+
+Every function named ``nvfp4_*`` here has the C signature of the same name in
+``include/nvfp4decode.h`` and returns its status (``NVFP4_OK`` = 0).  Device
+pointers and streams are plain integers (``tensor.data_ptr()``,
+``torch.cuda.current_stream().cuda_stream``).  The torch helpers at the end
+only allocate device memory and pass pointers; all compute runs in the
+library's CUDA kernels.  If the library is missing this module raises: there
+is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4decode.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4decode.h")
+
+NVFP4_OK = 0
+NVFP4_ERR_ARG = -1
+NVFP4_ERR_M = -2
+NVFP4_ERR_SHAPE = -3
+NVFP4_ERR_ALIGN = -4
+NVFP4_ERR_BAD_SCALE = -5
+NVFP4_ERR_CUDA = -6
+NVFP4_ERR_CAPTURE = -7
+NVFP4_ERR_DEVICE = -8
+NVFP4_DESC_GEMM = 0
+NVFP4_DESC_GATEUP_SILU = 1
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+_I = ctypes.c_int
+
+
+class Nvfp4GemmDesc(ctypes.Structure):
+    _fields_ = [("kind", _I), ("X", _P), ("wq", _P), ("ws", _P), ("gscale", _F),
+                ("wq2", _P), ("ws2", _P), ("gscale2", _F), ("out", _P), ("N", _I64), ("K", _I64)]
+
+
+_SIGNATURES = {
+    "nvfp4_packed_bytes": (_I, [_I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
+    "nvfp4_pack_check": (_I, [_P, _P, _I64, _I64, _P, _P, _P]),
+    "nvfp4_gemm_decode": (_I, [_P, _I, _P, _P, _F, _P, _I64, _I64, _P]),
+    "nvfp4_gemm_gateup_silu": (_I, [_P, _I, _P, _P, _F, _P, _P, _F, _P, _I64, _I64, _P]),
+    "nvfp4_round_create": (_I, [ctypes.POINTER(Nvfp4GemmDesc), _I, ctypes.POINTER(_P)]),
+    "nvfp4_round_nodes": (_I, [_P, ctypes.POINTER(_I)]),
+    "nvfp4_round_replay": (_I, [_P, _I, _P]),
+    "nvfp4_round_replay_host": (_I, [_P, _I, _P, _P, _SZ, _P, _P, _SZ, _P]),
+    "nvfp4_round_destroy": (_I, [_P]),
+    "nvfp4_dequant_debug": (_I, [_P, _P, _F, _P, _I64, _I64, _P]),
+    "nvfp4_unpack_debug": (_I, [_P, _P, _I64, _I64, _P, _P, _P]),
+    "nvfp4_host_dequant_unit": (_I, [_P, _P, _F, _P]),
+    "nvfp4_host_pack_unit": (_I, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
+    "nvfp4_status_string": (ctypes.c_char_p, [_I]),
+    "nvfp4_last_cuda_error": (_I, []),
+    "nvfp4_device_status": (_I, []),
+    "nvfp4_version": (_I, []),
+}
+
+_lib = None
+
+
+def load():
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with __graft_entry__.build()")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def header_functions():
+    """Names of the functions include/nvfp4decode.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)))
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        msg = status_string(status)
+        if status == NVFP4_ERR_CUDA:
+            msg += f" (cuda error {load().nvfp4_last_cuda_error()})"
+        super().__init__(f"{what}: {msg} [{status}]" if what else f"{msg} [{status}]")
+        self.status = status
+
+
+def status_string(status: int) -> str:
+    return load().nvfp4_status_string(int(status)).decode()
+
+
+def check(status: int, what: str = "") -> int:
+    if status != NVFP4_OK:
+        raise Nvfp4Error(status, what)
+    return status
+
+
+def _s(stream):
+    return None if stream is None else int(stream)
+
+
+# ------------------------------------------------------- raw C-ABI calls
+
+def nvfp4_packed_bytes(N, K):
+    """(status, wq_bytes, ws_bytes)."""
+    a, b = _SZ(), _SZ()
+    st = load().nvfp4_packed_bytes(int(N), int(K), ctypes.byref(a), ctypes.byref(b))
+    return st, a.value, b.value
+
+
+def nvfp4_pack_check(wq_canon, ws_canon, N, K, wq_dev, ws_dev, stream):
+    return load().nvfp4_pack_check(wq_canon, ws_canon, int(N), int(K), wq_dev, ws_dev, _s(stream))
+
+
+def nvfp4_gemm_decode(X, M, wq_dev, ws_dev, gscale, Y, N, K, stream):
+    return load().nvfp4_gemm_decode(X, int(M), wq_dev, ws_dev, float(gscale), Y, int(N), int(K),
+                                    _s(stream))
+
+
+def nvfp4_gemm_gateup_silu(X, M, wq_gate, ws_gate, gscale_gate, wq_up, ws_up, gscale_up, H, Nff, K,
+                           stream):
+    return load().nvfp4_gemm_gateup_silu(X, int(M), wq_gate, ws_gate, float(gscale_gate), wq_up,
+                                         ws_up, float(gscale_up), H, int(Nff), int(K), _s(stream))
+
+
+def nvfp4_round_create(descs):
+    """(status, handle) for a sequence of Nvfp4GemmDesc."""
+    arr = (Nvfp4GemmDesc * len(descs))(*descs)
+    h = _P()
+    st = load().nvfp4_round_create(arr, len(descs), ctypes.byref(h))
+    return st, h.value
+
+
+def nvfp4_round_nodes(handle):
+    n = _I()
+    st = load().nvfp4_round_nodes(handle, ctypes.byref(n))
+    return st, n.value
+
+
+def nvfp4_round_replay(handle, M, stream):
+    return load().nvfp4_round_replay(handle, int(M), _s(stream))
+
+
+def nvfp4_round_replay_host(handle, M, x_host, x_dev, x_bytes, y_dev, y_host, y_bytes, stream):
+    return load().nvfp4_round_replay_host(handle, int(M), x_host, x_dev, int(x_bytes), y_dev, y_host,
+                                          int(y_bytes), _s(stream))
+
+
+def nvfp4_round_destroy(handle):
+    return load().nvfp4_round_destroy(handle)
+
+
+def nvfp4_dequant_debug(wq_dev, ws_dev, gscale, W, N, K, stream):
+    return load().nvfp4_dequant_debug(wq_dev, ws_dev, float(gscale), W, int(N), int(K), _s(stream))
+
+
+def nvfp4_unpack_debug(wq_dev, ws_dev, N, K, wq_canon, ws_canon, stream):
+    return load().nvfp4_unpack_debug(wq_dev, ws_dev, int(N), int(K), wq_canon, ws_canon, _s(stream))
+
+
+def nvfp4_host_dequant_unit(q_unit, s_unit, gscale, W):
+    return load().nvfp4_host_dequant_unit(q_unit, s_unit, float(gscale), W)
+
+
+def nvfp4_host_pack_unit(wq_canon, ws_canon, N, K, tile, chunk, q_unit, s_unit):
+    return load().nvfp4_host_pack_unit(wq_canon, ws_canon, int(N), int(K), int(tile), int(chunk),
+                                       q_unit, s_unit)
+
+
+def nvfp4_status_string(status):
+    return status_string(status)
+
+
+def nvfp4_last_cuda_error():
+    return load().nvfp4_last_cuda_error()
+
+
+def nvfp4_device_status():
+    return load().nvfp4_device_status()
+
+
+def nvfp4_version():
+    return load().nvfp4_version()
+
+
+# ------------------------------------------------------- torch helpers
+
+def _stream_ptr(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def pack(q_canon, s_canon, stream=None):
+    """Pack canonical device planes (torch uint8 [N][K/2], [N][K/16]) into
+    freshly allocated device-layout planes; returns (wq_dev, ws_dev)."""
+    import torch
+    N, half_k = q_canon.shape
+    K = half_k * 2
+    st, nq, ns = nvfp4_packed_bytes(N, K)
+    check(st, "nvfp4_packed_bytes")
+    wq = torch.empty(nq, dtype=torch.uint8, device=q_canon.device)
+    ws = torch.empty(ns, dtype=torch.uint8, device=q_canon.device)
+    check(nvfp4_pack_check(q_canon.data_ptr(), s_canon.data_ptr(), N, K, wq.data_ptr(),
+                           ws.data_ptr(), _stream_ptr(stream)), "nvfp4_pack_check")
+    return wq, ws
+
+
+def gemm_decode(X, wq, ws, gscale, N, K, Y=None, stream=None):
+    """Y float32 [M][N] = gscale * X . dequant(W)^T (X: torch bf16 [M][K] on the device)."""
+    import torch
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    check(nvfp4_gemm_decode(X.data_ptr(), M, wq.data_ptr(), ws.data_ptr(), gscale, Y.data_ptr(), N,
+                            K, _stream_ptr(stream)), "nvfp4_gemm_decode")
+    return Y
+
+
+def gemm_gateup_silu(X, wq_g, ws_g, gscale_g, wq_u, ws_u, gscale_u, Nff, K, H=None, stream=None):
+    """H bf16 [M][Nff] = silu(X . Wg^T) * (X . Wu^T), one launch."""
+    import torch
+    M = X.shape[0]
+    if H is None:
+        H = torch.empty((M, Nff), dtype=torch.bfloat16, device=X.device)
+    check(nvfp4_gemm_gateup_silu(X.data_ptr(), M, wq_g.data_ptr(), ws_g.data_ptr(), gscale_g,
+                                 wq_u.data_ptr(), ws_u.data_ptr(), gscale_u, H.data_ptr(), Nff, K,
+                                 _stream_ptr(stream)), "nvfp4_gemm_gateup_silu")
+    return H
+
+
+def dequant_debug(wq, ws, gscale, N, K, stream=None):
+    import torch
+    W = torch.empty((N, K), dtype=torch.float32, device=wq.device)
+    check(nvfp4_dequant_debug(wq.data_ptr(), ws.data_ptr(), gscale, W.data_ptr(), N, K,
+                              _stream_ptr(stream)), "nvfp4_dequant_debug")
+    return W
+
+
+def unpack_debug(wq, ws, N, K, stream=None):
+    import torch
+    q = torch.empty((N, K // 2), dtype=torch.uint8, device=wq.device)
+    s = torch.empty((N, K // 16), dtype=torch.uint8, device=wq.device)
+    check(nvfp4_unpack_debug(wq.data_ptr(), ws.data_ptr(), N, K, q.data_ptr(), s.data_ptr(),
+                             _stream_ptr(stream)), "nvfp4_unpack_debug")
+    return q, s
+
+
+class Round:
+    """Owner of an nvfp4_round handle built from descriptors."""
+
+    def __init__(self, descs):
+        st, h = nvfp4_round_create(descs)
+        check(st, "nvfp4_round_create")
+        self.handle = h
+        self._descs = list(descs)
+
+    @property
+    def nodes(self):
+        st, n = nvfp4_round_nodes(self.handle)
+        check(st, "nvfp4_round_nodes")
+        return n
+
+    def replay(self, M, stream=None):
+        check(nvfp4_round_replay(self.handle, M, _stream_ptr(stream)), "nvfp4_round_replay")
+
+    def replay_host(self, M, x_host, x_dev, y_dev, y_host, stream=None):
+        """H2D copy of x_host -> x_dev, replay, D2H copy of y_dev -> y_host (torch tensors)."""
+        xb = x_host.numel() * x_host.element_size()
+        yb = y_host.numel() * y_host.element_size()
+        check(nvfp4_round_replay_host(self.handle, M, x_host.data_ptr(), x_dev.data_ptr(), xb,
+                                      y_dev.data_ptr(), y_host.data_ptr(), yb, _stream_ptr(stream)),
+              "nvfp4_round_replay_host")
+
+    def close(self):
+        if self.handle:
+            nvfp4_round_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def desc(kind, X, wq, ws, gscale, out, N, K, wq2=None, ws2=None, gscale2=0.0):
+    """An Nvfp4GemmDesc from torch tensors."""
+    return Nvfp4GemmDesc(kind, X.data_ptr(), wq.data_ptr(), ws.data_ptr(), float(gscale),
+                         wq2.data_ptr() if wq2 is not None else None,
+                         ws2.data_ptr() if ws2 is not None else None, float(gscale2),
+                         out.data_ptr(), int(N), int(K))

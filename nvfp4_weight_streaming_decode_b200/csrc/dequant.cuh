@@ -1,0 +1,63 @@
+// dequant.cuh -- device-side register dequantisation of one lane's share of
+// a 32 x 64 unit (see layout.cuh for the layout), and the bf16 tensor-core
+// step that consumes it.  Used by the GEMM kernels and by the dequant debug
+// export, so the exported weights are exactly the ones the GEMMs multiply.
+#pragma once
+#include <stdint.h>
+
+#include "layout.cuh"
+
+namespace nvfp4 {
+
+__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// The lane's four scales as broadcast bf16x2 pairs, each = e4m3 * 2^118:
+// S[r][0] for row 16r+g, S[r][1] for row 16r+g+8.
+__device__ __forceinline__ void scale_pairs(uint32_t sw, uint32_t (&S)[2][2])
+{
+    const uint32_t rows_hi = sw & 0xFF00FF00u;          // rows g+8 of groups 0, 1
+    const uint32_t rows_lo = (sw << 8) & 0xFF00FF00u;   // rows g of groups 0, 1
+    uint32_t p_lo = hmul2_bf16(hmul2_bf16(scale_raw_pair(rows_lo), kBf16Pow2_119x2), kBf16Pow2_119x2);
+    uint32_t p_hi = hmul2_bf16(hmul2_bf16(scale_raw_pair(rows_hi), kBf16Pow2_119x2), kBf16Pow2_119x2);
+    S[0][0] = prmt(p_lo, p_lo, 0x1010u);
+    S[0][1] = prmt(p_hi, p_hi, 0x1010u);
+    S[1][0] = prmt(p_lo, p_lo, 0x3232u);
+    S[1][1] = prmt(p_hi, p_hi, 0x3232u);
+}
+
+// A fragment (a0a1, a2a3, a4a5, a6a7) of code word w of row group r:
+// bf16x2 values e2m1 * e4m3 * 2^-8, exact.
+__device__ __forceinline__ void dequant_word(uint32_t w, const uint32_t (&S)[2][2], int r,
+                                             uint32_t (&a)[4])
+{
+    uint32_t c[4];
+    code_pairs(w, c);
+    a[0] = hmul2_bf16(c[0], S[r][0]);
+    a[1] = hmul2_bf16(c[1], S[r][1]);
+    a[2] = hmul2_bf16(c[2], S[r][0]);
+    a[3] = hmul2_bf16(c[3], S[r][1]);
+}
+
+// d += A(16x16, bf16) . B(16x8, bf16), FP32 accumulation.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+}  // namespace nvfp4

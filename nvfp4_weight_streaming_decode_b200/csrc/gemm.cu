@@ -1,0 +1,579 @@
+// gemm.cu -- the NVFP4 decode GEMM kernels for sm_100a and their launch.
+//
+// Y[M][N] = gscale * X[M][K] . dequant(W)^T for M = 1..8 lanes (ignis
+// README, "The decode round": all lanes share one pass over the weights,
+// which streams at the card's memory bandwidth), and the fused gate/up
+// variant H = bf16(silu(Xg) * Xu) that reads both projections in the same
+// pass.
+//
+// Work split ("stream-K"): the matrix is a sequence of 32 x 64 units stored
+// contiguously in tile-major order.  Every warp of the grid takes one
+// contiguous range of units -- one contiguous run of bytes in each weight
+// plane -- so all warps stream nearly the same number of bytes whatever N
+// and K are.  A warp pulls its range through a private ring of shared-memory
+// stages with 1-D bulk copies (the TMA engine, no tensor map, no multicast),
+// one mbarrier per stage, dequantises in registers and feeds bf16 m16n8k16
+// tensor-core MMAs with the lanes of X as the 8-wide N side.  A tile
+// (32 rows) that straddles warp ranges is finished by whichever of its
+// contributors arrives last: each writes its partial sums to the workspace,
+// bumps the tile's counter, and the last one adds the partials in warp order
+// (fixed, so results are bit-identical run to run) and runs the epilogue.
+// No thread ever waits on another warp or CTA.
+//
+// PDL: every kernel signals its dependents at entry, issues its weight
+// copies (which depend on nothing), and only then waits for the preceding
+// grid before it reads X or touches outputs and workspace.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "dequant.cuh"
+#include "internal.h"
+#include "layout.cuh"
+
+namespace nvfp4 {
+
+__device__ unsigned int g_device_status;
+
+constexpr int kWarps = 8;                  // warps per CTA
+constexpr int kSlotFloats = 512;           // partial-sum slot: 2 matrices x 32 rows x 8 lanes
+constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls before giving up
+
+struct KParams {
+    const uint8_t* wq[2];
+    const uint8_t* ws[2];
+    float gs[2];
+    const uint16_t* X;
+    void* out;
+    long long N, K, k_chunks, units;
+    long long total_warps;
+    float* partials;
+    unsigned* counters;
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// All 32 lanes poll; gives up (returns false) after kWaitLimit rounds.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity)
+{
+    for (uint32_t it = 0; it < kWaitLimit; ++it)
+        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    return false;
+}
+
+__device__ __forceinline__ uint64_t evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                          uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+        : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float4 ld_cg_f4(const float* p)
+{
+    float4 v;
+    asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ long long range_begin(long long units, long long tw, long long w)
+{
+    return units * w / tw;
+}
+
+// Warp whose range holds unit x.
+__device__ __forceinline__ long long range_owner(long long units, long long tw, long long x)
+{
+    return ((x + 1) * tw - 1) / units;
+}
+
+template <int M, int NW>
+__device__ __forceinline__ void epilogue(const KParams& p, long long tile, const float (&acc)[NW][2][4],
+                                         int g, int t)
+{
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = 2 * t + (i & 1);
+            const long long n = tile * kTileN + 16 * r + g + ((i & 2) ? 8 : 0);
+            if (m < M && n < p.N) {
+                if (NW == 1) {
+                    static_cast<float*>(p.out)[m * p.N + n] = (acc[0][r][i] * kEpilogueScale) * p.gs[0];
+                } else {
+                    const float gv = (acc[0][r][i] * kEpilogueScale) * p.gs[0];
+                    const float uv = (acc[NW - 1][r][i] * kEpilogueScale) * p.gs[1];
+                    const float h = gv / (1.0f + expf(-gv)) * uv;
+                    static_cast<__nv_bfloat16*>(p.out)[m * p.N + n] = __float2bfloat16_rn(h);
+                }
+            }
+        }
+}
+
+template <int M, int NW, int STAGES>
+__global__ void __launch_bounds__(kWarps * 32)
+decode_gemm_kernel(const KParams p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int kStage = NW * kUnitBytes;
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const long long gw = (long long)blockIdx.x * kWarps + warp;
+
+    // Dependents may begin launching; they wait for this grid before using its results.
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    const long long U = p.units, TW = p.total_warps, KC = p.k_chunks;
+    const long long u0 = range_begin(U, TW, gw), u1 = range_begin(U, TW, gw + 1);
+    if (u0 >= u1) return;
+
+    uint8_t* ring = smem + warp * (STAGES * kStage);
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t bar_s = smem_addr(smem + kWarps * STAGES * kStage) + warp * STAGES * 8;
+
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(bar_s + 8 * s);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+
+    const uint64_t pol = evict_first_policy();
+    auto issue = [&](long long u, int st) {
+        const uint32_t dst = ring_s + st * kStage;
+        const uint32_t bar = bar_s + 8 * st;
+        mbar_expect_tx(bar, kStage);
+#pragma unroll
+        for (int mat = 0; mat < NW; ++mat) {
+            bulk_load(dst + mat * kUnitBytes, p.wq[mat] + u * kUnitQ, kUnitQ, bar, pol);
+            bulk_load(dst + mat * kUnitBytes + kUnitQ, p.ws[mat] + u * kUnitS, kUnitS, bar, pol);
+        }
+    };
+
+    const long long n_units = u1 - u0;
+    if (lane == 0) {
+        const long long npre = n_units < STAGES ? n_units : STAGES;
+        for (long long i = 0; i < npre; ++i) issue(u0 + i, (int)i);
+    }
+
+    // Everything below reads X or writes outputs / workspace: wait for the producer grid.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    float acc[NW][2][4];
+#pragma unroll
+    for (int a = 0; a < NW; ++a)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[a][r][i] = 0.f;
+
+    auto flush = [&](long long tile) {
+        const long long ts = tile * KC, te = ts + KC;
+        if (ts >= u0 && te <= u1) {
+            epilogue<M, NW>(p, tile, acc, g, t);
+            return;
+        }
+        const int slot = (u0 / KC == tile) ? 0 : 1;
+        float* dst = p.partials + ((size_t)gw * 2 + slot) * kSlotFloats + lane * (NW * 8);
+#pragma unroll
+        for (int a = 0; a < NW; ++a)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                reinterpret_cast<float4*>(dst)[a * 2 + r] =
+                    make_float4(acc[a][r][0], acc[a][r][1], acc[a][r][2], acc[a][r][3]);
+        __threadfence();
+        __syncwarp();
+        const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
+        unsigned count = 0;
+        for (long long w = glo; w <= ghi; ++w)
+            count += range_begin(U, TW, w) < range_begin(U, TW, w + 1) ? 1u : 0u;
+        unsigned last = 0;
+        if (lane == 0) last = (atomicAdd(&p.counters[glo], 1u) == count - 1u) ? 1u : 0u;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) return;
+        __threadfence();
+        float sum[NW][2][4];
+#pragma unroll
+        for (int a = 0; a < NW; ++a)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
+        for (long long w = glo; w <= ghi; ++w) {
+            const long long wb = range_begin(U, TW, w);
+            if (wb >= range_begin(U, TW, w + 1)) continue;
+            const int ws = (wb / KC == tile) ? 0 : 1;
+            const float* src = p.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8);
+#pragma unroll
+            for (int a = 0; a < NW; ++a)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const float4 v = ld_cg_f4(src + (a * 2 + r) * 4);
+                    sum[a][r][0] += v.x;
+                    sum[a][r][1] += v.y;
+                    sum[a][r][2] += v.z;
+                    sum[a][r][3] += v.w;
+                }
+        }
+        epilogue<M, NW>(p, tile, sum, g, t);
+        if (lane == 0) atomicExch(&p.counters[glo], 0u);
+    };
+
+    long long cur_tile = u0 / KC;
+    for (long long i = 0; i < n_units; ++i) {
+        const long long u = u0 + i;
+        const int st = (int)(i % STAGES);
+        const uint32_t parity = (uint32_t)((i / STAGES) & 1);
+        if (!warp_wait(bar_s + 8 * st, parity)) {
+            // Give up: flag it, then wait (bounded) for the copies still in flight.
+            if (lane == 0) atomicOr(&g_device_status, 1u);
+            for (long long j = i + 1; j < n_units && j < i + STAGES; ++j)
+                warp_wait(bar_s + 8 * (int)(j % STAGES), (uint32_t)((j / STAGES) & 1));
+            return;
+        }
+        const long long tile = u / KC;
+        const long long chunk = u - tile * KC;
+        if (tile != cur_tile) {
+            flush(cur_tile);
+#pragma unroll
+            for (int a = 0; a < NW; ++a)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc[a][r][k] = 0.f;
+            cur_tile = tile;
+        }
+
+        // This lane's 16 columns of X for lane row g (zeros past M or past K).
+        uint32_t xw[8];
+        const long long col = chunk * kChunkK + 16 * t;
+        if (g < M && col < p.K) {
+            const uint16_t* xp = p.X + (long long)g * p.K + col;
+            const uint4 lo = ld_nc_v4(xp), hi = ld_nc_v4(xp + 8);
+            xw[0] = lo.x; xw[1] = lo.y; xw[2] = lo.z; xw[3] = lo.w;
+            xw[4] = hi.x; xw[5] = hi.y; xw[6] = hi.z; xw[7] = hi.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) xw[k] = 0u;
+        }
+
+        const uint8_t* stage = ring + st * kStage;
+#pragma unroll
+        for (int mat = 0; mat < NW; ++mat) {
+            const uint8_t* sb = stage + mat * kUnitBytes;
+            const uint4 q0 = *reinterpret_cast<const uint4*>(sb + 16 * lane);
+            const uint4 q1 = *reinterpret_cast<const uint4*>(sb + 512 + 16 * lane);
+            const uint32_t sw = *reinterpret_cast<const uint32_t*>(sb + kUnitQ + 4 * lane);
+            const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+            uint32_t S[2][2];
+            scale_pairs(sw, S);
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    uint32_t a[4];
+                    dequant_word(q[4 * r + s], S, r, a);
+                    mma_bf16_16816(acc[mat][r], a, xw[2 * s], xw[2 * s + 1]);
+                }
+        }
+
+        // The MMAs above consumed every word read from this stage, so the
+        // stage can be refilled.
+        __syncwarp();
+        if (lane == 0 && i + STAGES < n_units) issue(u + STAGES, st);
+    }
+    flush(cur_tile);
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+
+constexpr int kStagesPlain = 5;
+constexpr int kStagesFused = 3;
+
+template <int M, int NW>
+struct KernelOf {
+    static constexpr int stages = NW == 1 ? kStagesPlain : kStagesFused;
+    static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages>; }
+    static size_t smem() { return (size_t)kWarps * stages * (NW * kUnitBytes + 8); }
+};
+
+struct KernelInfo {
+    void* fn = nullptr;
+    size_t smem = 0;
+    int blocks_per_sm = 0;  // filled on first use
+};
+
+template <int NW>
+KernelInfo kernel_info_for(int M)
+{
+    KernelInfo k;
+    switch (M) {
+#define NVFP4_CASE(m)                        \
+    case m:                                  \
+        k.fn = KernelOf<m, NW>::fn();        \
+        k.smem = KernelOf<m, NW>::smem();    \
+        break;
+        NVFP4_CASE(1) NVFP4_CASE(2) NVFP4_CASE(3) NVFP4_CASE(4)
+        NVFP4_CASE(5) NVFP4_CASE(6) NVFP4_CASE(7) NVFP4_CASE(8)
+#undef NVFP4_CASE
+    }
+    return k;
+}
+
+std::mutex g_mu;
+DeviceState g_states[64];
+KernelInfo g_kernels[64][2][kMaxM];  // [device][kind][M-1]
+
+}  // namespace
+
+int device_state(cudaStream_t stream, DeviceState** out)
+{
+    int dev = 0;
+    NVFP4_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return NVFP4_ERR_ARG;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& s = g_states[dev];
+    if (s.device == dev) {
+        *out = &s;
+        return NVFP4_OK;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    NVFP4_CUDA_TRY(cudaStreamIsCapturing(stream, &cs));
+    if (cs != cudaStreamCaptureStatusNone) return NVFP4_ERR_CAPTURE;
+    int sms = 0;
+    NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    int max_threads = 0;
+    NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&max_threads, cudaDevAttrMaxThreadsPerMultiProcessor, dev));
+    const int max_warps = sms * (max_threads / 32);
+    float* partials = nullptr;
+    unsigned* counters = nullptr;
+    NVFP4_CUDA_TRY(cudaMalloc(&partials, (size_t)max_warps * 2 * kSlotFloats * sizeof(float)));
+    cudaError_t e = cudaMalloc(&counters, (size_t)max_warps * sizeof(unsigned));
+    if (e != cudaSuccess) {
+        cudaFree(partials);
+        return fail_cuda(e);
+    }
+    e = cudaMemset(counters, 0, (size_t)max_warps * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        cudaFree(partials);
+        cudaFree(counters);
+        return fail_cuda(e);
+    }
+    s.sm_count = sms;
+    s.max_warps = max_warps;
+    s.partials = partials;
+    s.counters = counters;
+    s.device = dev;
+    *out = &s;
+    return NVFP4_OK;
+}
+
+static int kernel_for(int dev, int kind, int M, KernelInfo** out)
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    KernelInfo& k = g_kernels[dev][kind][M - 1];
+    if (k.blocks_per_sm == 0) {
+        KernelInfo fresh = kind == 0 ? kernel_info_for<1>(M) : kernel_info_for<2>(M);
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(fresh.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)fresh.smem));
+        int nb = 0;
+        NVFP4_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fresh.fn, kWarps * 32,
+                                                                     fresh.smem));
+        if (nb < 1) return NVFP4_ERR_CUDA;
+        fresh.blocks_per_sm = nb;
+        k = fresh;
+    }
+    *out = &k;
+    return NVFP4_OK;
+}
+
+int prepare_kernel(DeviceState* ds, int kind, int M)
+{
+    KernelInfo* k = nullptr;
+    return kernel_for(ds->device, kind, M, &k);
+}
+
+int validate_gemm(const GemmArgs& a)
+{
+    if (a.kind != 0 && a.kind != 1) return NVFP4_ERR_ARG;
+    const int nw = a.kind == 0 ? 1 : 2;
+    if (!a.X || !a.out) return NVFP4_ERR_ARG;
+    for (int i = 0; i < nw; ++i)
+        if (!a.wq[i] || !a.ws[i]) return NVFP4_ERR_ARG;
+    int st = check_m(a.M);
+    if (st != NVFP4_OK) return st;
+    st = check_shape(a.N, a.K);
+    if (st != NVFP4_OK) return st;
+    if (!aligned16(a.X) || !aligned16(a.out)) return NVFP4_ERR_ALIGN;
+    for (int i = 0; i < nw; ++i)
+        if (!aligned16(a.wq[i]) || !aligned16(a.ws[i])) return NVFP4_ERR_ALIGN;
+    return NVFP4_OK;
+}
+
+int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* ds)
+{
+    KernelInfo* k = nullptr;
+    int st = kernel_for(ds->device, a.kind, a.M, &k);
+    if (st != NVFP4_OK) return st;
+    const Geometry geo = geometry(a.N, a.K);
+    long long ctas = (long long)ds->sm_count * k->blocks_per_sm;
+    const long long need = (geo.units + kWarps - 1) / kWarps;
+    if (need < ctas) ctas = need;
+    if (ctas * kWarps > ds->max_warps) ctas = ds->max_warps / kWarps;
+
+    KParams p;
+    const int nw = a.kind == 0 ? 1 : 2;
+    for (int i = 0; i < 2; ++i) {
+        p.wq[i] = a.wq[i < nw ? i : 0];
+        p.ws[i] = a.ws[i < nw ? i : 0];
+        p.gs[i] = a.gscale[i < nw ? i : 0];
+    }
+    p.X = static_cast<const uint16_t*>(a.X);
+    p.out = a.out;
+    p.N = a.N;
+    p.K = a.K;
+    p.k_chunks = geo.k_chunks;
+    p.units = geo.units;
+    p.total_warps = ctas * kWarps;
+    p.partials = ds->partials;
+    p.counters = ds->counters;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = k->smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    void* args[] = {&p};
+    NVFP4_CUDA_TRY(cudaLaunchKernelExC(&cfg, k->fn, args));
+    return NVFP4_OK;
+}
+
+int read_and_clear_device_status(int* status)
+{
+    unsigned v = 0;
+    NVFP4_CUDA_TRY(cudaDeviceSynchronize());
+    NVFP4_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_device_status, sizeof v));
+    if (v != 0) {
+        const unsigned zero = 0;
+        NVFP4_CUDA_TRY(cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero));
+        int dev = 0;
+        NVFP4_CUDA_TRY(cudaGetDevice(&dev));
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (dev >= 0 && dev < 64 && g_states[dev].device == dev)
+            NVFP4_CUDA_TRY(cudaMemset(g_states[dev].counters, 0,
+                                      (size_t)g_states[dev].max_warps * sizeof(unsigned)));
+        NVFP4_CUDA_TRY(cudaDeviceSynchronize());
+    }
+    *status = (int)v;
+    return NVFP4_OK;
+}
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
+                                 float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream)
+{
+    GemmArgs a = {};
+    a.kind = 0;
+    a.X = X;
+    a.M = M;
+    a.wq[0] = wq_dev;
+    a.ws[0] = ws_dev;
+    a.gscale[0] = gscale;
+    a.out = Y;
+    a.N = N;
+    a.K = K;
+    int st = validate_gemm(a);
+    if (st != NVFP4_OK) return st;
+    DeviceState* ds = nullptr;
+    st = device_state((cudaStream_t)stream, &ds);
+    if (st != NVFP4_OK) return st;
+    return launch_gemm(a, (cudaStream_t)stream, false, ds);
+}
+
+extern "C" int nvfp4_gemm_gateup_silu(const void* X, int M, const uint8_t* wq_gate,
+                                      const uint8_t* ws_gate, float gscale_gate, const uint8_t* wq_up,
+                                      const uint8_t* ws_up, float gscale_up, void* H, int64_t Nff,
+                                      int64_t K, nvfp4_stream_t stream)
+{
+    GemmArgs a = {};
+    a.kind = 1;
+    a.X = X;
+    a.M = M;
+    a.wq[0] = wq_gate;
+    a.ws[0] = ws_gate;
+    a.gscale[0] = gscale_gate;
+    a.wq[1] = wq_up;
+    a.ws[1] = ws_up;
+    a.gscale[1] = gscale_up;
+    a.out = H;
+    a.N = Nff;
+    a.K = K;
+    int st = validate_gemm(a);
+    if (st != NVFP4_OK) return st;
+    DeviceState* ds = nullptr;
+    st = device_state((cudaStream_t)stream, &ds);
+    if (st != NVFP4_OK) return st;
+    return launch_gemm(a, (cudaStream_t)stream, false, ds);
+}

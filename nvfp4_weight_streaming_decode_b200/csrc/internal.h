@@ -1,0 +1,62 @@
+// internal.h -- host-side plumbing shared by the library's translation units:
+// status handling, argument checks, per-device state and the launch hooks
+// the round builder uses.  Not part of the C ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nvfp4decode.h"
+#include "layout.cuh"
+
+namespace nvfp4 {
+
+// Remember a failed CUDA call for nvfp4_last_cuda_error() and map it to a status.
+int fail_cuda(cudaError_t e);
+#define NVFP4_CUDA_TRY(expr)                          \
+    do {                                              \
+        cudaError_t e_ = (expr);                      \
+        if (e_ != cudaSuccess) return ::nvfp4::fail_cuda(e_); \
+    } while (0)
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int check_shape(int64_t N, int64_t K);
+int check_m(int M);
+
+struct Geometry {
+    int64_t n_tiles, k_chunks, units;
+};
+Geometry geometry(int64_t N, int64_t K);
+
+// Per-device state: SM count, split-K workspace and counters.  Created by
+// the first call on a device, which must not be inside a stream capture.
+struct DeviceState {
+    int device = -1;
+    int sm_count = 0;
+    int max_warps = 0;        // capacity of the workspace, in warps
+    float* partials = nullptr;
+    unsigned* counters = nullptr;
+};
+int device_state(cudaStream_t stream, DeviceState** out);
+
+// Launch one decode GEMM (kind 0) or fused gate/up (kind 1).  `pdl` marks the
+// launch as a programmatic dependent of the previous work on the stream.
+struct GemmArgs {
+    int kind;
+    const void* X;
+    int M;
+    const uint8_t* wq[2];
+    const uint8_t* ws[2];
+    float gscale[2];
+    void* out;
+    int64_t N, K;
+};
+int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* ds);
+int validate_gemm(const GemmArgs& a);
+// Resolve a kernel variant (attributes, occupancy) ahead of a stream capture.
+int prepare_kernel(DeviceState* ds, int kind, int M);
+
+// Device-side status word (nonzero after a bounded wait gave up).
+int read_and_clear_device_status(int* status);
+
+}  // namespace nvfp4

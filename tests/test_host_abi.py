@@ -1,0 +1,128 @@
+"""CPU tests of the C-ABI library: symbols, argument checks, and the host
+model of the device layout against the oracle.  No GPU and no kernel launch:
+every call here returns before the library touches CUDA."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+from nvfp4_weight_streaming_decode_b200 import abi, synth
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__  # noqa: F401  (build helpers)
+    from nvfp4_weight_streaming_decode_b200 import build
+    build.build()
+    return abi.load()
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def test_library_exports_every_header_symbol(lib):
+    names = abi.header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(abi._SIGNATURES) == set(names)
+
+
+def test_status_strings(lib):
+    for st in range(-8, 1):
+        assert abi.status_string(st)
+    assert "unknown" in abi.status_string(-99)
+    assert abi.nvfp4_version() >= 100
+
+
+@pytest.mark.parametrize("N,K,ok", [(1, 16, True), (5120, 5120, True), (0, 16, False), (8, 8, False),
+                                    (8, 24, False), (-1, 64, False)])
+def test_packed_bytes(lib, N, K, ok):
+    st, nq, ns = abi.nvfp4_packed_bytes(N, K)
+    if not ok:
+        assert st == abi.NVFP4_ERR_SHAPE
+        return
+    assert st == abi.NVFP4_OK
+    units = -(-N // 32) * -(-K // 64)
+    assert nq == units * 1024 and ns == units * 128
+
+
+def test_argument_errors_return_before_any_cuda_call(lib):
+    p = 1 << 20  # a fake, aligned "device" pointer: never dereferenced on these paths
+    assert abi.nvfp4_gemm_decode(p, 0, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_gemm_decode(p, 9, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_gemm_decode(p, 1, p, p, 1.0, p, 32, 40, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_gemm_decode(p, 1, p, p, 1.0, p, 0, 64, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_gemm_decode(None, 1, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_gemm_decode(p + 8, 1, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_decode(p, 1, p + 4, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_decode(p, 1, p, p, 1.0, p + 2, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_gateup_silu(p, 1, p, p, 1.0, None, p, 1.0, p, 32, 64, None) == \
+        abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_gemm_gateup_silu(p, 10, p, p, 1.0, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_pack_check(None, p, 32, 64, p, p, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_pack_check(p, p, 32, 63, p, p, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_pack_check(p, p, 32, 64, p + 1, p, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_dequant_debug(p, p, 1.0, p + 4, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_round_replay(None, 1, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_round_destroy(None) == abi.NVFP4_OK
+    bad = abi.Nvfp4GemmDesc(7, p, p, p, 1.0, None, None, 0.0, p, 32, 64)
+    st, h = abi.nvfp4_round_create([bad])
+    assert st == abi.NVFP4_ERR_ARG and not h
+    badm = abi.Nvfp4GemmDesc(0, p, p, p, 1.0, None, None, 0.0, p, 32, 40)
+    assert abi.nvfp4_round_create([badm])[0] == abi.NVFP4_ERR_SHAPE
+
+
+def _host_dequant(q, s, gscale):
+    """Dequantise a whole matrix through the library's host model, unit by unit."""
+    N, K = q.shape[0], q.shape[1] * 2
+    nt, kc = -(-N // 32), -(-K // 64)
+    W = np.zeros((nt * 32, kc * 64), np.float32)
+    qu = np.zeros(1024, np.uint8)
+    su = np.zeros(128, np.uint8)
+    Wu = np.zeros((32, 64), np.float32)
+    for tile in range(nt):
+        for chunk in range(kc):
+            abi.check(abi.nvfp4_host_pack_unit(_ptr(q), _ptr(s), N, K, tile, chunk, _ptr(qu), _ptr(su)))
+            abi.check(abi.nvfp4_host_dequant_unit(_ptr(qu), _ptr(su), gscale, _ptr(Wu)))
+            W[tile * 32:(tile + 1) * 32, chunk * 64:(chunk + 1) * 64] = Wu
+    return W[:N, :K], W
+
+
+@pytest.mark.parametrize("N,K", [(32, 64), (256, 512), (45, 80), (7, 16), (33, 208)])
+def test_host_layout_model_dequant_is_bit_exact(lib, N, K):
+    q, s = synth.matrix(20, N * 7 + K, N, K)
+    W, Wfull = _host_dequant(q, s, 1.0 / 64)
+    ref = oracle.dequant(q, s, 1.0 / 64)
+    assert np.array_equal(W.view(np.uint32), ref.view(np.uint32))
+    # padding rows and columns dequantise to zero
+    pad = Wfull.copy()
+    pad[:N, :K] = 0
+    assert not np.any(pad)
+
+
+def test_host_layout_model_special_scales(lib):
+    N, K = 32, 128
+    q, s = synth.matrix(21, 0, N, K)
+    specials = [0x00, 0x80, 0x01, 0x07, 0x08, 0x7E, 0xFE, 0xB9, 0x81, 0x3F]
+    for i, b in enumerate(specials):
+        s[i % N, i % (K // 16)] = b
+    for gscale in (1.0, 1.0 / 64, 3.0, -0.5):
+        W, _ = _host_dequant(q, s, gscale)
+        ref = oracle.dequant(q, s, gscale)
+        assert np.array_equal(W.view(np.uint32), ref.view(np.uint32)), gscale
+
+
+def test_host_layout_model_every_code_with_every_scale(lib):
+    # rows cycle the 254 non-NaN scale codes, columns cycle the 16 element codes
+    scales = np.array([b for b in range(256) if (b & 0x7F) != 0x7F], np.uint8)
+    N, K = 256, 64
+    q = np.zeros((N, K // 2), np.uint8)
+    codes = np.arange(K) % 16
+    q[:] = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    s = np.repeat(scales[np.arange(N) % scales.size][:, None], K // 16, axis=1).astype(np.uint8)
+    W, _ = _host_dequant(q, s, 1.0)
+    ref = oracle.dequant(q, s, 1.0)
+    assert np.array_equal(W.view(np.uint32), ref.view(np.uint32))
