@@ -15,7 +15,8 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libnvfp4decode.so")
+# NVFP4_LIB may name another build of the same library (same ABI).
+LIB_PATH = os.environ.get("NVFP4_LIB") or os.path.join(HERE, "libnvfp4decode.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4decode.h")
 
 NVFP4_OK = 0

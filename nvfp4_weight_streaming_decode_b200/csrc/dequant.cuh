@@ -23,6 +23,21 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
     return r;
 }
 
+// {lo, lo} and {hi, hi} of a bf16x2 (the multiply can take these as operand
+// swizzles).
+__device__ __forceinline__ uint32_t bcast_lo(uint32_t p)
+{
+    uint32_t r;
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n mov.b32 %0, {l, l};\n}" : "=r"(r) : "r"(p));
+    return r;
+}
+__device__ __forceinline__ uint32_t bcast_hi(uint32_t p)
+{
+    uint32_t r;
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n mov.b32 %0, {h, h};\n}" : "=r"(r) : "r"(p));
+    return r;
+}
+
 // The lane's four scales as broadcast bf16x2 pairs, each = e4m3 * 2^118:
 // S[r][0] for row 16r+g, S[r][1] for row 16r+g+8.
 __device__ __forceinline__ void scale_pairs(uint32_t sw, uint32_t (&S)[2][2])
@@ -31,10 +46,10 @@ __device__ __forceinline__ void scale_pairs(uint32_t sw, uint32_t (&S)[2][2])
     const uint32_t rows_lo = (sw << 8) & 0xFF00FF00u;   // rows g of groups 0, 1
     uint32_t p_lo = hmul2_bf16(hmul2_bf16(scale_raw_pair(rows_lo), kBf16Pow2_119x2), kBf16Pow2_119x2);
     uint32_t p_hi = hmul2_bf16(hmul2_bf16(scale_raw_pair(rows_hi), kBf16Pow2_119x2), kBf16Pow2_119x2);
-    S[0][0] = prmt(p_lo, p_lo, 0x1010u);
-    S[0][1] = prmt(p_hi, p_hi, 0x1010u);
-    S[1][0] = prmt(p_lo, p_lo, 0x3232u);
-    S[1][1] = prmt(p_hi, p_hi, 0x3232u);
+    S[0][0] = bcast_lo(p_lo);
+    S[0][1] = bcast_lo(p_hi);
+    S[1][0] = bcast_hi(p_lo);
+    S[1][1] = bcast_hi(p_hi);
 }
 
 // A fragment (a0a1, a2a3, a4a5, a6a7) of code word w of row group r:

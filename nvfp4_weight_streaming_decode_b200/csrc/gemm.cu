@@ -38,6 +38,7 @@ namespace nvfp4 {
 __device__ unsigned int g_device_status;
 
 constexpr int kWarps = 8;                  // warps per CTA
+constexpr int kMinBlocks = 2;              // CTAs per SM the register budget is sized for
 constexpr int kSlotFloats = 512;           // partial-sum slot: 2 matrices x 32 rows x 8 lanes
 constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls before giving up
 
@@ -116,6 +117,19 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p)
     return v;
 }
 
+// 32 bytes of X (two 16-byte loads) when `pred`, zeros otherwise; no branch.
+__device__ __forceinline__ void ld_x32(const void* p, bool pred, uint32_t (&x)[8])
+{
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.u32 q, %9, 0;\n"
+        " mov.b32 %0, 0; mov.b32 %1, 0; mov.b32 %2, 0; mov.b32 %3, 0;\n"
+        " mov.b32 %4, 0; mov.b32 %5, 0; mov.b32 %6, 0; mov.b32 %7, 0;\n"
+        " @q ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%8];\n"
+        " @q ld.global.nc.v4.u32 {%4,%5,%6,%7}, [%8+16];\n}"
+        : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7])
+        : "l"(p), "r"((uint32_t)pred));
+}
+
 __device__ __forceinline__ float4 ld_cg_f4(const float* p)
 {
     float4 v;
@@ -136,9 +150,18 @@ __device__ __forceinline__ long long range_owner(long long units, long long tw, 
     return ((x + 1) * tw - 1) / units;
 }
 
+// Output side of a kernel, passed by value to the out-of-line tile finisher.
+struct OutArgs {
+    void* out;
+    float* partials;
+    unsigned* counters;
+    long long N, units, total_warps, k_chunks;
+    float gs0, gs1;
+};
+
 template <int M, int NW>
-__device__ __forceinline__ void epilogue(const KParams& p, long long tile, const float (&acc)[NW][2][4],
-                                         int g, int t)
+__device__ __forceinline__ void epilogue(const OutArgs& o, long long tile, const float (&acc)[NW][2][4], int g,
+                                         int t)
 {
 #pragma unroll
     for (int r = 0; r < 2; ++r)
@@ -146,25 +169,118 @@ __device__ __forceinline__ void epilogue(const KParams& p, long long tile, const
         for (int i = 0; i < 4; ++i) {
             const int m = 2 * t + (i & 1);
             const long long n = tile * kTileN + 16 * r + g + ((i & 2) ? 8 : 0);
-            if (m < M && n < p.N) {
+            if (m < M && n < o.N) {
                 if (NW == 1) {
-                    static_cast<float*>(p.out)[m * p.N + n] = (acc[0][r][i] * kEpilogueScale) * p.gs[0];
+                    static_cast<float*>(o.out)[m * o.N + n] = (acc[0][r][i] * kEpilogueScale) * o.gs0;
                 } else {
-                    const float gv = (acc[0][r][i] * kEpilogueScale) * p.gs[0];
-                    const float uv = (acc[NW - 1][r][i] * kEpilogueScale) * p.gs[1];
+                    const float gv = (acc[0][r][i] * kEpilogueScale) * o.gs0;
+                    const float uv = (acc[NW - 1][r][i] * kEpilogueScale) * o.gs1;
                     const float h = gv / (1.0f + expf(-gv)) * uv;
-                    static_cast<__nv_bfloat16*>(p.out)[m * p.N + n] = __float2bfloat16_rn(h);
+                    static_cast<__nv_bfloat16*>(o.out)[m * o.N + n] = __float2bfloat16_rn(h);
                 }
             }
         }
 }
 
-template <int M, int NW, int STAGES>
-__global__ void __launch_bounds__(kWarps * 32)
+// One lane's share of a unit: X fragments are in xw; sq and ss point at the
+// lane's code bytes and scale word in shared memory.  Adds the unit's products into acc.
+__device__ __forceinline__ void mma_unit(const uint8_t* sq, const uint8_t* ss, const uint32_t (&xw)[8],
+                                         float (&acc)[2][4])
+{
+    const uint4 q0 = *reinterpret_cast<const uint4*>(sq);
+    const uint4 q1 = *reinterpret_cast<const uint4*>(sq + 512);
+    const uint32_t sw = *reinterpret_cast<const uint32_t*>(ss);
+    const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    uint32_t S[2][2];
+    scale_pairs(sw, S);
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            uint32_t a[4];
+            dequant_word(q[4 * r + s], S, r, a);
+            mma_bf16_16816(acc[r], a, xw[2 * s], xw[2 * s + 1]);
+        }
+}
+
+// Load one contributor's partial sums (this lane's NW*8 floats).
+template <int NW>
+__device__ __forceinline__ void load_partial(const float* src, float4 (&v)[NW * 2])
+{
+#pragma unroll
+    for (int k = 0; k < NW * 2; ++k) v[k] = ld_cg_f4(src + 4 * k);
+}
+
+// End of a tile for this warp.  The warp has already stored its sums in its
+// partial slot.  A tile the warp covered alone goes straight to the
+// epilogue; otherwise the warp counts itself in, and the last contributor
+// adds every partial in warp order (glo..ghi, a fixed order, so the result
+// does not depend on who arrives last) and runs the epilogue.  Out of line,
+// so the streaming loop does not carry its registers.
+template <int M, int NW>
+__device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane)
+{
+    const long long U = o.units, TW = o.total_warps, KC = o.k_chunks;
+    const long long ts = tile * KC, te = ts + KC;
+    const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
+    float sum[NW][2][4];
+    if (glo != ghi) {
+        __threadfence();
+        __syncwarp();
+        // Every warp below total_warps has a non-empty range, so the
+        // contributors are exactly the warps glo..ghi.
+        unsigned last = 0;
+        if (lane == 0) last = (atomicAdd(&o.counters[glo], 1u) == (unsigned)(ghi - glo)) ? 1u : 0u;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) return;
+        __threadfence();
+    }
+    const int glo_slot = (range_begin(U, TW, glo) >= ts) ? 0 : 1;
+#pragma unroll
+    for (int a = 0; a < NW; ++a)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
+    constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together
+    for (long long w0 = glo; w0 <= ghi; w0 += kBatch) {
+        float4 v[kBatch][NW * 2];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const long long w = w0 + b;
+            if (w <= ghi) {
+                const int ws = (w == glo) ? glo_slot : 0;
+                load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            if (w0 + b <= ghi) {
+#pragma unroll
+                for (int a = 0; a < NW; ++a)
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        sum[a][r][0] += v[b][a * 2 + r].x;
+                        sum[a][r][1] += v[b][a * 2 + r].y;
+                        sum[a][r][2] += v[b][a * 2 + r].z;
+                        sum[a][r][3] += v[b][a * 2 + r].w;
+                    }
+            }
+        }
+    }
+    epilogue<M, NW>(o, tile, sum, lane >> 2, lane & 3);
+    if (glo != ghi && lane == 0) atomicExch(&o.counters[glo], 0u);
+}
+
+// STAGES shared-memory stages per warp, each holding UPS consecutive units of
+// each of the NW matrices (one bulk copy per plane and matrix per stage).
+template <int M, int NW, int STAGES, int UPS>
+__global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
 decode_gemm_kernel(const KParams p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int kStage = NW * kUnitBytes;
+    constexpr int kMatStage = UPS * kUnitBytes;
+    constexpr int kStage = NW * kMatStage;
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -175,8 +291,10 @@ decode_gemm_kernel(const KParams p)
     asm volatile("griddepcontrol.launch_dependents;");
 
     const long long U = p.units, TW = p.total_warps, KC = p.k_chunks;
+    if (gw >= TW) return;
     const long long u0 = range_begin(U, TW, gw), u1 = range_begin(U, TW, gw + 1);
-    if (u0 >= u1) return;
+    const int n_units = (int)(u1 - u0);
+    const int n_stages = (n_units + UPS - 1) / UPS;
 
     uint8_t* ring = smem + warp * (STAGES * kStage);
     const uint32_t ring_s = smem_addr(ring);
@@ -190,21 +308,23 @@ decode_gemm_kernel(const KParams p)
     __syncwarp();
 
     const uint64_t pol = evict_first_policy();
-    auto issue = [&](long long u, int st) {
-        const uint32_t dst = ring_s + st * kStage;
-        const uint32_t bar = bar_s + 8 * st;
-        mbar_expect_tx(bar, kStage);
+    auto issue = [&](int j, int slot) {
+        const long long ub = u0 + (long long)j * UPS;
+        const int rem = n_units - j * UPS;
+        const int cnt = rem < UPS ? rem : UPS;
+        const uint32_t dst = ring_s + slot * kStage;
+        const uint32_t bar = bar_s + 8 * slot;
+        mbar_expect_tx(bar, (uint32_t)(NW * cnt * kUnitBytes));
 #pragma unroll
         for (int mat = 0; mat < NW; ++mat) {
-            bulk_load(dst + mat * kUnitBytes, p.wq[mat] + u * kUnitQ, kUnitQ, bar, pol);
-            bulk_load(dst + mat * kUnitBytes + kUnitQ, p.ws[mat] + u * kUnitS, kUnitS, bar, pol);
+            bulk_load(dst + mat * kMatStage, p.wq[mat] + ub * kUnitQ, cnt * kUnitQ, bar, pol);
+            bulk_load(dst + mat * kMatStage + UPS * kUnitQ, p.ws[mat] + ub * kUnitS, cnt * kUnitS, bar, pol);
         }
     };
 
-    const long long n_units = u1 - u0;
     if (lane == 0) {
-        const long long npre = n_units < STAGES ? n_units : STAGES;
-        for (long long i = 0; i < npre; ++i) issue(u0 + i, (int)i);
+        const int npre = n_stages < STAGES ? n_stages : STAGES;
+        for (int j = 0; j < npre; ++j) issue(j, j);
     }
 
     // Everything below reads X or writes outputs / workspace: wait for the producer grid.
@@ -218,136 +338,111 @@ decode_gemm_kernel(const KParams p)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[a][r][i] = 0.f;
 
-    auto flush = [&](long long tile) {
-        const long long ts = tile * KC, te = ts + KC;
-        if (ts >= u0 && te <= u1) {
-            epilogue<M, NW>(p, tile, acc, g, t);
-            return;
-        }
-        const int slot = (u0 / KC == tile) ? 0 : 1;
-        float* dst = p.partials + ((size_t)gw * 2 + slot) * kSlotFloats + lane * (NW * 8);
-#pragma unroll
-        for (int a = 0; a < NW; ++a)
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-                reinterpret_cast<float4*>(dst)[a * 2 + r] =
-                    make_float4(acc[a][r][0], acc[a][r][1], acc[a][r][2], acc[a][r][3]);
-        __threadfence();
-        __syncwarp();
-        const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
-        unsigned count = 0;
-        for (long long w = glo; w <= ghi; ++w)
-            count += range_begin(U, TW, w) < range_begin(U, TW, w + 1) ? 1u : 0u;
-        unsigned last = 0;
-        if (lane == 0) last = (atomicAdd(&p.counters[glo], 1u) == count - 1u) ? 1u : 0u;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) return;
-        __threadfence();
-        float sum[NW][2][4];
-#pragma unroll
-        for (int a = 0; a < NW; ++a)
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
-        for (long long w = glo; w <= ghi; ++w) {
-            const long long wb = range_begin(U, TW, w);
-            if (wb >= range_begin(U, TW, w + 1)) continue;
-            const int ws = (wb / KC == tile) ? 0 : 1;
-            const float* src = p.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8);
-#pragma unroll
-            for (int a = 0; a < NW; ++a)
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const float4 v = ld_cg_f4(src + (a * 2 + r) * 4);
-                    sum[a][r][0] += v.x;
-                    sum[a][r][1] += v.y;
-                    sum[a][r][2] += v.z;
-                    sum[a][r][3] += v.w;
-                }
-        }
-        epilogue<M, NW>(p, tile, sum, g, t);
-        if (lane == 0) atomicExch(&p.counters[glo], 0u);
-    };
-
-    long long cur_tile = u0 / KC;
-    for (long long i = 0; i < n_units; ++i) {
-        const long long u = u0 + i;
-        const int st = (int)(i % STAGES);
-        const uint32_t parity = (uint32_t)((i / STAGES) & 1);
-        if (!warp_wait(bar_s + 8 * st, parity)) {
+    long long tile = u0 / KC;
+    const long long first_tile = tile;
+    int chunk = (int)(u0 - tile * KC);
+    const int kc_last = (int)KC - 1;
+    const int K32 = (int)p.K;
+    // X row of this lane (row 0 stands in past M; those lanes load nothing)
+    const uint16_t* xp = p.X + (long long)(g < M ? g : 0) * p.K + chunk * kChunkK + 16 * t;
+    int col = chunk * kChunkK + 16 * t;                 // this lane's first column in the unit
+    const bool x_lane = g < M;
+    const uint32_t q_off = 16 * lane, s_off = 4 * lane;
+    int slot = 0;
+    uint32_t parity = 0;
+    int i = 0;                                          // units consumed
+    for (int j = 0; j < n_stages; ++j) {
+        if (!warp_wait(bar_s + 8 * slot, parity)) {
             // Give up: flag it, then wait (bounded) for the copies still in flight.
             if (lane == 0) atomicOr(&g_device_status, 1u);
-            for (long long j = i + 1; j < n_units && j < i + STAGES; ++j)
-                warp_wait(bar_s + 8 * (int)(j % STAGES), (uint32_t)((j / STAGES) & 1));
+            int s2 = slot;
+            uint32_t p2 = parity;
+            for (int j2 = j; j2 < n_stages && j2 < j + STAGES; ++j2) {
+                warp_wait(bar_s + 8 * s2, p2);
+                if (++s2 == STAGES) {
+                    s2 = 0;
+                    p2 ^= 1u;
+                }
+            }
             return;
         }
-        const long long tile = u / KC;
-        const long long chunk = u - tile * KC;
-        if (tile != cur_tile) {
-            flush(cur_tile);
+        const uint8_t* stage = ring + slot * kStage;
 #pragma unroll
-            for (int a = 0; a < NW; ++a)
+        for (int v = 0; v < UPS; ++v) {
+            if (i < n_units) {
+                // This lane's 16 columns of X for lane row g (zeros past M or past K).
+                uint32_t xw[8];
+                ld_x32(xp, x_lane && col < K32, xw);
+                const uint8_t* sq = stage + v * kUnitQ + q_off;
+                const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
 #pragma unroll
-                for (int r = 0; r < 2; ++r)
+                for (int mat = 0; mat < NW; ++mat) mma_unit(sq + mat * kMatStage, ss + mat * kMatStage, xw, acc[mat]);
+                ++i;
+                const bool tile_end = chunk == kc_last;
+                if (tile_end || i == n_units) {
+                    // Partial slot: 0 for the tile this warp's range starts in, 1 for a later one.
+                    const int slot_id = (tile == first_tile) ? 0 : 1;
+                    float* dst = p.partials + ((size_t)gw * 2 + slot_id) * kSlotFloats + lane * (NW * 8);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) acc[a][r][k] = 0.f;
-            cur_tile = tile;
-        }
-
-        // This lane's 16 columns of X for lane row g (zeros past M or past K).
-        uint32_t xw[8];
-        const long long col = chunk * kChunkK + 16 * t;
-        if (g < M && col < p.K) {
-            const uint16_t* xp = p.X + (long long)g * p.K + col;
-            const uint4 lo = ld_nc_v4(xp), hi = ld_nc_v4(xp + 8);
-            xw[0] = lo.x; xw[1] = lo.y; xw[2] = lo.z; xw[3] = lo.w;
-            xw[4] = hi.x; xw[5] = hi.y; xw[6] = hi.z; xw[7] = hi.w;
-        } else {
+                    for (int a = 0; a < NW; ++a)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) xw[k] = 0u;
-        }
-
-        const uint8_t* stage = ring + st * kStage;
+                        for (int r = 0; r < 2; ++r)
+                            reinterpret_cast<float4*>(dst)[a * 2 + r] =
+                                make_float4(acc[a][r][0], acc[a][r][1], acc[a][r][2], acc[a][r][3]);
+                    OutArgs o;
+                    o.out = p.out;
+                    o.partials = p.partials;
+                    o.counters = p.counters;
+                    o.N = p.N;
+                    o.units = p.units;
+                    o.total_warps = p.total_warps;
+                    o.k_chunks = p.k_chunks;
+                    o.gs0 = p.gs[0];
+                    o.gs1 = p.gs[1];
+                    tile_done<M, NW>(o, tile, lane);
 #pragma unroll
-        for (int mat = 0; mat < NW; ++mat) {
-            const uint8_t* sb = stage + mat * kUnitBytes;
-            const uint4 q0 = *reinterpret_cast<const uint4*>(sb + 16 * lane);
-            const uint4 q1 = *reinterpret_cast<const uint4*>(sb + 512 + 16 * lane);
-            const uint32_t sw = *reinterpret_cast<const uint32_t*>(sb + kUnitQ + 4 * lane);
-            const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-            uint32_t S[2][2];
-            scale_pairs(sw, S);
+                    for (int a = 0; a < NW; ++a)
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+                        for (int r = 0; r < 2; ++r)
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    uint32_t a[4];
-                    dequant_word(q[4 * r + s], S, r, a);
-                    mma_bf16_16816(acc[mat][r], a, xw[2 * s], xw[2 * s + 1]);
+                            for (int k = 0; k < 4; ++k) acc[a][r][k] = 0.f;
                 }
+                if (tile_end) {
+                    ++tile;
+                    chunk = 0;
+                    col = 16 * t;
+                    xp -= kc_last * kChunkK;                 // back to column 16t of the same row
+                } else {
+                    ++chunk;
+                    col += kChunkK;
+                    xp += kChunkK;
+                }
+            }
         }
-
         // The MMAs above consumed every word read from this stage, so the
         // stage can be refilled.
         __syncwarp();
-        if (lane == 0 && i + STAGES < n_units) issue(u + STAGES, st);
+        if (lane == 0 && j + STAGES < n_stages) issue(j + STAGES, slot);
+        if (++slot == STAGES) {
+            slot = 0;
+            parity ^= 1u;
+        }
     }
-    flush(cur_tile);
 }
 
 // ------------------------------------------------------------------ host side
 
 namespace {
 
-constexpr int kStagesPlain = 5;
-constexpr int kStagesFused = 3;
+constexpr int kStagesPlain = 3, kUnitsPerStagePlain = 4;
+constexpr int kStagesFused = 3, kUnitsPerStageFused = 2;
 
 template <int M, int NW>
 struct KernelOf {
     static constexpr int stages = NW == 1 ? kStagesPlain : kStagesFused;
-    static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages>; }
-    static size_t smem() { return (size_t)kWarps * stages * (NW * kUnitBytes + 8); }
+    static constexpr int ups = NW == 1 ? kUnitsPerStagePlain : kUnitsPerStageFused;
+    static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages, ups>; }
+    static size_t smem() { return (size_t)kWarps * stages * (NW * ups * kUnitBytes + 8); }
 };
 
 struct KernelInfo {
@@ -474,6 +569,9 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
     const long long need = (geo.units + kWarps - 1) / kWarps;
     if (need < ctas) ctas = need;
     if (ctas * kWarps > ds->max_warps) ctas = ds->max_warps / kWarps;
+    // Never more warps than units: every warp below total_warps gets a
+    // non-empty range (the split-K combine relies on it).
+    const long long total_warps = ctas * kWarps < geo.units ? ctas * kWarps : geo.units;
 
     KParams p;
     const int nw = a.kind == 0 ? 1 : 2;
@@ -488,7 +586,7 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
     p.K = a.K;
     p.k_chunks = geo.k_chunks;
     p.units = geo.units;
-    p.total_warps = ctas * kWarps;
+    p.total_warps = total_warps;
     p.partials = ds->partials;
     p.counters = ds->counters;
 

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/nvfp4decode.h"
+#include "nvfp4decode.h"
 #include "layout.cuh"
 
 namespace nvfp4 {
