@@ -117,6 +117,17 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p)
     return v;
 }
 
+// 32 bytes of X into x when `pred`; x keeps its contents otherwise.
+__device__ __forceinline__ void ld_x32_keep(const void* p, bool pred, uint32_t (&x)[8])
+{
+    asm(
+        "{\n .reg .pred q;\n setp.ne.u32 q, %9, 0;\n"
+        " @q ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%8];\n"
+        " @q ld.global.nc.v4.u32 {%4,%5,%6,%7}, [%8+16];\n}"
+        : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]), "+r"(x[7])
+        : "l"(p), "r"((uint32_t)pred));
+}
+
 // 32 bytes of X (two 16-byte loads) when `pred`, zeros otherwise; no branch.
 __device__ __forceinline__ void ld_x32(const void* p, bool pred, uint32_t (&x)[8])
 {
@@ -351,6 +362,7 @@ decode_gemm_kernel(const KParams p)
     int slot = 0;
     uint32_t parity = 0;
     int i = 0;                                          // units consumed
+    uint32_t xf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // fast-path X (stays zero past M)
     for (int j = 0; j < n_stages; ++j) {
         if (!warp_wait(bar_s + 8 * slot, parity)) {
             // Give up: flag it, then wait (bounded) for the copies still in flight.
@@ -367,7 +379,24 @@ decode_gemm_kernel(const KParams p)
             return;
         }
         const uint8_t* stage = ring + slot * kStage;
+        if (n_units - i > UPS && kc_last - chunk >= UPS) {
+            // Fast path: a full stage inside one tile that reaches neither the
+            // tile's last chunk nor the end of the warp's range, so no unit
+            // needs a bounds, tile-end or range-end check.
 #pragma unroll
+            for (int v = 0; v < UPS; ++v) {
+                ld_x32_keep(xp + v * kChunkK, x_lane, xf);
+                const uint8_t* sq = stage + v * kUnitQ + q_off;
+                const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
+#pragma unroll
+                for (int mat = 0; mat < NW; ++mat) mma_unit(sq + mat * kMatStage, ss + mat * kMatStage, xf, acc[mat]);
+            }
+            i += UPS;
+            chunk += UPS;
+            col += UPS * kChunkK;
+            xp += UPS * kChunkK;
+        } else {
+#pragma unroll 1
         for (int v = 0; v < UPS; ++v) {
             if (i < n_units) {
                 // This lane's 16 columns of X for lane row g (zeros past M or past K).
@@ -418,6 +447,7 @@ decode_gemm_kernel(const KParams p)
                     xp += kChunkK;
                 }
             }
+        }
         }
         // The MMAs above consumed every word read from this stage, so the
         // stage can be refilled.
