@@ -37,8 +37,8 @@ namespace nvfp4 {
 
 __device__ unsigned int g_device_status;
 
-constexpr int kWarps = 8;                  // warps per CTA
-constexpr int kMinBlocks = 2;              // CTAs per SM the register budget is sized for
+constexpr int kWarps = 16;                 // warps per CTA: one CTA per SM, so every warp has equal priority
+constexpr int kMinBlocks = 1;              // CTAs per SM the register budget is sized for
 constexpr int kSlotFloats = 512;           // partial-sum slot: 2 matrices x 32 rows x 8 lanes
 constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls before giving up
 
@@ -253,7 +253,7 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
-    constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together
+    constexpr int kBatch = NW == 1 ? 8 : 2;  // contributors whose loads are in flight together
     for (long long w0 = glo; w0 <= ghi; w0 += kBatch) {
         float4 v[kBatch][NW * 2];
 #pragma unroll
