@@ -45,6 +45,10 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="only warm-up and timed replays (for an ncu launch list)")
+    ap.add_argument("--gemm-case", default=None, choices=["head", "proj", "gateup", "down"],
+                    help="only three direct calls of one workload GEMM at --width (for an ncu capture)")
     return ap.parse_args()
 
 
@@ -170,33 +174,32 @@ def max_over_ranks(value, world):
 # ------------------------------------------------------------------ CPU oracle legs
 
 def oracle_sample(device, seconds_budget):
-    """Time the float64 oracle on a bounded row sample of layer 0's q/k/v GEMM
-    (K = 5120, M = 8); returns (GB/s of weights processed, cores, description)."""
+    """Time the float64 oracle on a bounded sample of the round's layer-0 q/k/v
+    GEMM (K = 5120, M = 8): blocks of rows, cycling through the matrix, until
+    the time budget is spent; returns (GB/s of weights processed, cores,
+    description)."""
     import numpy as np
+    import torch
 
     import oracle
     from nvfp4_weight_streaming_decode_b200 import synth
     hidden = synth.WORKLOADS[4]["hidden"]
     q_full, s_full = synth.torch_matrix(4, 0, 3 * hidden, hidden, device)
-    X = synth.torch_activations(4, 0, 8, hidden, device)
-    Xb = X.view(__import__("torch").int16).cpu().numpy().view(np.uint16)
-    rows_total = 0
-    elapsed = 0.0
-    r = 16
-    while True:
-        rows = min(r, q_full.shape[0])
-        q = q_full[:rows].cpu().numpy()
-        s = s_full[:rows].cpu().numpy()
+    q_full, s_full = q_full.cpu().numpy(), s_full.cpu().numpy()
+    Xb = synth.torch_activations(4, 0, 8, hidden, device).view(torch.int16).cpu().numpy().view(np.uint16)
+    block = 1024
+    rows_total, elapsed, lo = 0, 0.0, 0
+    while elapsed < seconds_budget:
+        q = np.ascontiguousarray(q_full[lo:lo + block])
+        s = np.ascontiguousarray(s_full[lo:lo + block])
         t0 = time.perf_counter()
         oracle.gemm(Xb, q, s, synth.GSCALE)
-        dt = time.perf_counter() - t0
-        rows_total += rows
-        elapsed += dt
-        if elapsed >= seconds_budget or rows == q_full.shape[0]:
-            break
-        r = int(min(q_full.shape[0], max(2 * r, r * (seconds_budget - elapsed) / max(dt, 1e-3) * 0.5)))
+        elapsed += time.perf_counter() - t0
+        rows_total += q.shape[0]
+        lo = (lo + block) % q_full.shape[0]
     gbs = rows_total * hidden * (0.5 + 1 / 16) / elapsed / 1e9
-    return gbs, oracle.threads(), f"oracle GEMM, M=8, {rows_total} rows of layer-0 q/k/v (K={hidden}) in {elapsed:.1f} s"
+    return gbs, oracle.threads(), (f"float64 oracle GEMM, M=8, {rows_total} rows (blocks of {block}, cycling) "
+                                   f"of the round's layer-0 q/k/v matrix, K={hidden}, {elapsed:.1f} s")
 
 
 def run_reference(args):
@@ -211,7 +214,7 @@ def run_reference(args):
     hidden = synth.WORKLOADS[4]["hidden"]
     q_full, s_full = synth.matrix(4, 0, 3 * hidden, hidden)
     Xb = synth.activations(synth.rng(4, 0), args.width, hidden)
-    per_step_rows = 128
+    per_step_rows = 2048
     times = []
     rows_done = 0
     for i in range(args.warmup + args.steps):
@@ -246,82 +249,70 @@ def run_reference(args):
 # ------------------------------------------------------------------ GPU legs
 
 def gemm_sweep(dev, hbm_peak):
-    """Standalone decode GEMMs per workload and width; CUDA events over
-    back-to-back launches with enough rotating weight copies to exceed L2."""
+    """Single decode GEMMs per workload and width, timed on the device: each
+    case is a chain of back-to-back launches captured as a C-ABI round (one
+    graph, PDL between nodes), rotating through enough weight copies to
+    exceed L2, and replayed under CUDA events."""
     import torch
 
     from nvfp4_weight_streaming_decode_b200 import abi, synth
     from nvfp4_weight_streaming_decode_b200.workloads import BYTES_PER_WEIGHT, make_matrix
     out = []
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.Stream(device=dev)
+    G, D = abi.NVFP4_DESC_GEMM, abi.NVFP4_DESC_GATEUP_SILU
 
-    def time_calls(fn, n_iter, copies):
-        for i in range(3):
-            fn(i % copies)
+    def time_chain(descs, reps=10):
+        rnd = abi.Round(descs)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                rnd.replay(8, stream)
         torch.cuda.synchronize()
+        res = {}
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(n_iter):
-            fn(i % copies)
-        e1.record(stream)
-        e1.synchronize()
-        return e0.elapsed_time(e1) / n_iter * 1e-3
+        for M in range(1, 9):
+            with torch.cuda.stream(stream):
+                rnd.replay(M, stream)
+                e0.record(stream)
+                for _ in range(reps):
+                    rnd.replay(M, stream)
+                e1.record(stream)
+            e1.synchronize()
+            res[M] = e0.elapsed_time(e1) * 1e-3 / reps / len(descs)
+        rnd.close()
+        return res
 
-    # single projection N = K = 5120, 16 copies (236 MB > L2)
+    def add(name, t_by_m, wbytes, io):
+        for M, t in t_by_m.items():
+            b = wbytes + io(M)
+            out.append({"workload": name, "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
+                        "frac": b / t / 1e9 / hbm_peak})
+
+    X = synth.torch_activations(1, 8, 8, 17408, dev)
+    # single projection N = K = 5120: 16 copies (236 MB > L2), 32 nodes
     mats = [make_matrix(1, 500 + c, 5120, 5120, dev) for c in range(16)]
-    for M in range(1, 9):
-        X = synth.torch_activations(1, M, M, 5120, dev)
-        Y = torch.empty((M, 5120), dtype=torch.float32, device=dev)
-
-        def f(c, M=M, X=X, Y=Y):
-            m = mats[c]
-            abi.check(abi.nvfp4_gemm_decode(X.data_ptr(), M, m.wq.data_ptr(), m.ws.data_ptr(), synth.GSCALE,
-                                            Y.data_ptr(), 5120, 5120, stream.cuda_stream))
-        t = time_calls(f, 200, len(mats))
-        b = 5120 * 5120 * BYTES_PER_WEIGHT + 2 * M * 5120 + 4 * M * 5120
-        out.append({"workload": "proj_n5120_k5120", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
-                    "frac": b / t / 1e9 / hbm_peak})
+    Y = torch.empty((8, 5120), dtype=torch.float32, device=dev)
+    descs = [abi.desc(G, X, m.wq, m.ws, synth.GSCALE, Y, 5120, 5120) for m in mats + mats]
+    add("proj_n5120_k5120", time_chain(descs), 5120 * 5120 * BYTES_PER_WEIGHT,
+        lambda M: 2 * M * 5120 + 4 * M * 5120)
     del mats
-    # head N = 151936, K = 5120 (438 MB > L2)
+    # head N = 151936, K = 5120 (438 MB > L2), 4 nodes
     head = make_matrix(3, 0, 151936, 5120, dev, synth.EXP_LOGU_M6_4)
-    for M in (1, 4, 8):
-        X = synth.torch_activations(3, M, M, 5120, dev)
-        Y = torch.empty((M, 151936), dtype=torch.float32, device=dev)
-
-        def f(c, M=M, X=X, Y=Y):
-            abi.check(abi.nvfp4_gemm_decode(X.data_ptr(), M, head.wq.data_ptr(), head.ws.data_ptr(),
-                                            synth.GSCALE, Y.data_ptr(), 151936, 5120, stream.cuda_stream))
-        t = time_calls(f, 30, 1)
-        b = 151936 * 5120 * BYTES_PER_WEIGHT + 2 * M * 5120 + 4 * M * 151936
-        out.append({"workload": "head_n151936_k5120", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
-                    "frac": b / t / 1e9 / hbm_peak})
+    Yh = torch.empty((8, 151936), dtype=torch.float32, device=dev)
+    descs = [abi.desc(G, X, head.wq, head.ws, synth.GSCALE, Yh, 151936, 5120)] * 4
+    add("head_n151936_k5120", time_chain(descs, 5), 151936 * 5120 * BYTES_PER_WEIGHT,
+        lambda M: 2 * M * 5120 + 4 * M * 151936)
     del head
-    # fused MLP: gate/up 2 x 17408 x 5120 then down 5120 x 17408, 2 copies (300 MB > L2)
+    # fused MLP: gate/up 2 x 17408 x 5120 and down 5120 x 17408, 2 copies (300 MB > L2)
     sets = [(make_matrix(2, 600 + 3 * c, 17408, 5120, dev), make_matrix(2, 601 + 3 * c, 17408, 5120, dev),
              make_matrix(2, 602 + 3 * c, 5120, 17408, dev)) for c in range(2)]
-    for M in (1, 8):
-        X = synth.torch_activations(2, M, M, 5120, dev)
-        H = torch.empty((M, 17408), dtype=torch.bfloat16, device=dev)
-        Y = torch.empty((M, 5120), dtype=torch.float32, device=dev)
-
-        def fg(c, M=M, X=X, H=H):
-            g, u, _ = sets[c]
-            abi.check(abi.nvfp4_gemm_gateup_silu(X.data_ptr(), M, g.wq.data_ptr(), g.ws.data_ptr(), synth.GSCALE,
-                                                 u.wq.data_ptr(), u.ws.data_ptr(), synth.GSCALE, H.data_ptr(),
-                                                 17408, 5120, stream.cuda_stream))
-
-        def fd(c, M=M, H=H, Y=Y):
-            d = sets[c][2]
-            abi.check(abi.nvfp4_gemm_decode(H.data_ptr(), M, d.wq.data_ptr(), d.ws.data_ptr(), synth.GSCALE,
-                                            Y.data_ptr(), 5120, 17408, stream.cuda_stream))
-        t = time_calls(fg, 60, 2)
-        b = 2 * 17408 * 5120 * BYTES_PER_WEIGHT + 2 * M * 5120 + 2 * M * 17408
-        out.append({"workload": "mlp_gateup_2x17408_k5120", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
-                    "frac": b / t / 1e9 / hbm_peak})
-        t = time_calls(fd, 60, 2)
-        b = 5120 * 17408 * BYTES_PER_WEIGHT + 2 * M * 17408 + 4 * M * 5120
-        out.append({"workload": "mlp_down_n5120_k17408", "M": M, "us": t * 1e6, "GBps": b / t / 1e9,
-                    "frac": b / t / 1e9 / hbm_peak})
+    H = torch.empty((8, 17408), dtype=torch.bfloat16, device=dev)
+    descs = [abi.desc(D, X, g.wq, g.ws, synth.GSCALE, H, 17408, 5120, u.wq, u.ws, synth.GSCALE)
+             for (g, u, _) in sets + sets]
+    add("mlp_gateup_2x17408_k5120", time_chain(descs), 2 * 17408 * 5120 * BYTES_PER_WEIGHT,
+        lambda M: 2 * M * 5120 + 2 * M * 17408)
+    descs = [abi.desc(G, X, d.wq, d.ws, synth.GSCALE, Y, 5120, 17408) for (_, _, d) in sets + sets]
+    add("mlp_down_n5120_k17408", time_chain(descs), 5120 * 17408 * BYTES_PER_WEIGHT,
+        lambda M: 2 * M * 17408 + 4 * M * 5120)
     del sets
     torch.cuda.synchronize()
     return out
@@ -335,6 +326,32 @@ def round_io_bytes(r, M):
         m0 = r.mats[mkeys[0]]
         total += 2 * M * m0.K + (4 if kind == abi.NVFP4_DESC_GEMM else 2) * M * m0.N
     return total
+
+
+def run_gemm_case(args):
+    """Three direct nvfp4_gemm_decode / nvfp4_gemm_gateup_silu calls on one workload matrix."""
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi, build, synth
+    from nvfp4_weight_streaming_decode_b200.workloads import make_matrix
+    build.build()
+    dev = torch.device("cuda", 0)
+    M = args.width
+    shapes = {"head": (151936, 5120, synth.EXP_LOGU_M6_4), "proj": (5120, 5120, synth.EXP_UNIFORM_M4_2),
+              "gateup": (17408, 5120, synth.EXP_UNIFORM_M4_2), "down": (5120, 17408, synth.EXP_UNIFORM_M4_2)}
+    N, K, exp = shapes[args.gemm_case]
+    m = make_matrix(3, 0, N, K, dev, exp)
+    X = synth.torch_activations(3, 1, M, K, dev)
+    if args.gemm_case == "gateup":
+        u = make_matrix(3, 1, N, K, dev, exp)
+        for _ in range(3):
+            abi.gemm_gateup_silu(X, m.wq, m.ws, synth.GSCALE, u.wq, u.ws, synth.GSCALE, N, K)
+    else:
+        for _ in range(3):
+            abi.gemm_decode(X, m.wq, m.ws, synth.GSCALE, N, K)
+    torch.cuda.synchronize()
+    print(json.dumps({"gemm_case": args.gemm_case, "M": M, "N": N, "K": K, "ok": True}))
+    return 0
 
 
 def run_ours(args):
@@ -366,8 +383,10 @@ def run_ours(args):
 
     # per-width round times (detail): 20 replays each
     by_width = {}
+    if args.profile:
+        args.no_sweep = args.no_cpu_baseline = True
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for m in range(1, 9):
+    for m in (range(1, 9) if not args.profile else ()):
         with torch.cuda.stream(stream):
             for _ in range(3):
                 rnd.replay(m, stream)
@@ -402,7 +421,7 @@ def run_ours(args):
     x_host = torch.empty((M, w["hidden"]), dtype=torch.bfloat16).pin_memory()
     x_host.copy_(r.bufs["x0"][:M].cpu())
     y_host = torch.empty((M, w["vocab"]), dtype=torch.float32).pin_memory()
-    e2e_steps = max(10, args.steps // 4)
+    e2e_steps = max(10, args.steps // 4) if not args.profile else 1
     with torch.cuda.stream(stream):
         for _ in range(3):
             rnd.replay_host(M, x_host, r.bufs["x0"], r.bufs["logits"][:M], y_host, stream)
@@ -451,6 +470,7 @@ def run_ours(args):
             "round_ms": ms_per_step,
             "round_ms_by_width": by_width,
             "round_GBps_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 for m, t in by_width.items()},
+            "round_frac_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 / hbm_peak for m, t in by_width.items()},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_host.numel() * 2,
@@ -470,6 +490,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.gemm_case:
+        return run_gemm_case(args)
     return run_ours(args)
 
 
