@@ -57,7 +57,8 @@ enum {
     NVFP4_ERR_BAD_SCALE = -5, /* a scale byte is an E4M3 NaN code (0x7F / 0xFF) */
     NVFP4_ERR_CUDA = -6,      /* a CUDA runtime call failed; see nvfp4_last_cuda_error() */
     NVFP4_ERR_CAPTURE = -7,   /* first use of a device while its stream is being captured */
-    NVFP4_ERR_DEVICE = -8     /* a kernel's bounded wait gave up; see nvfp4_device_status() */
+    NVFP4_ERR_DEVICE = -8,    /* a kernel's bounded wait gave up; see nvfp4_device_status() */
+    NVFP4_ERR_SCRATCH = -9    /* the call needs more scratch than nvfp4_gemm_decode_noalloc's array holds */
 };
 
 /*
@@ -99,6 +100,34 @@ NVFP4_API int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon,
  */
 NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                       float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);
+
+/*
+ * The decode GEMM of nvfp4_gemm_decode, for callers that must not allocate
+ * device memory.  (No counterpart in the pages; it exists for callers.)
+ *
+ * nvfp4_gemm_decode allocates its split-K workspace with cudaMalloc on the
+ * first call on each device.  Some callers cannot allow that: an engine that
+ * reserves its whole device-memory plan at load time and forbids any later
+ * allocation, a plugin whose host application owns all device memory, or a
+ * latency-critical path that cannot take cudaMalloc's implicit device
+ * synchronisation.  This entry point calls no cudaMalloc, cudaFree or other
+ * allocating routine: its scratch (the split-K partial sums and arrival
+ * counters) is a file-scope static device array of this library, 10 MiB of
+ * partial sums plus 10 KiB of counters, enough for 2,560 warps; every GPU
+ * that loads the library holds it until the process exits.
+ *
+ * Arguments, layout and result are those of nvfp4_gemm_decode (the same
+ * kernel runs).  The first call on a device resolves the array's device
+ * address (cudaGetSymbolAddress) with that device current, so make that first
+ * call before any stream capture.  Each call clears the arrival counters on
+ * `stream` before the kernel.  All calls share the one array, which keeps the
+ * previous call's contents: calls that overlap on the GPU (other streams,
+ * other host threads) race on it and must be serialised by the caller.
+ * Returns NVFP4_ERR_SCRATCH if the launch would need more warps than the array
+ * holds (a device with more than 160 SMs).
+ */
+NVFP4_API int nvfp4_gemm_decode_noalloc(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
+                                        float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);
 
 /*
  * Fused MLP front half, asynchronous, one launch for both projections:

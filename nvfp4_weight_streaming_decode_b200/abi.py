@@ -28,6 +28,7 @@ NVFP4_ERR_BAD_SCALE = -5
 NVFP4_ERR_CUDA = -6
 NVFP4_ERR_CAPTURE = -7
 NVFP4_ERR_DEVICE = -8
+NVFP4_ERR_SCRATCH = -9
 NVFP4_DESC_GEMM = 0
 NVFP4_DESC_GATEUP_SILU = 1
 
@@ -47,6 +48,7 @@ _SIGNATURES = {
     "nvfp4_packed_bytes": (_I, [_I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
     "nvfp4_pack_check": (_I, [_P, _P, _I64, _I64, _P, _P, _P]),
     "nvfp4_gemm_decode": (_I, [_P, _I, _P, _P, _F, _P, _I64, _I64, _P]),
+    "nvfp4_gemm_decode_noalloc": (_I, [_P, _I, _P, _P, _F, _P, _I64, _I64, _P]),
     "nvfp4_gemm_gateup_silu": (_I, [_P, _I, _P, _P, _F, _P, _P, _F, _P, _I64, _I64, _P]),
     "nvfp4_round_create": (_I, [ctypes.POINTER(Nvfp4GemmDesc), _I, ctypes.POINTER(_P)]),
     "nvfp4_round_nodes": (_I, [_P, ctypes.POINTER(_I)]),
@@ -127,6 +129,12 @@ def nvfp4_pack_check(wq_canon, ws_canon, N, K, wq_dev, ws_dev, stream):
 def nvfp4_gemm_decode(X, M, wq_dev, ws_dev, gscale, Y, N, K, stream):
     return load().nvfp4_gemm_decode(X, int(M), wq_dev, ws_dev, float(gscale), Y, int(N), int(K),
                                     _s(stream))
+
+
+def nvfp4_gemm_decode_noalloc(X, M, wq_dev, ws_dev, gscale, Y, N, K, stream):
+    """nvfp4_gemm_decode without any device allocation (static scratch array in the library)."""
+    return load().nvfp4_gemm_decode_noalloc(X, int(M), wq_dev, ws_dev, float(gscale), Y, int(N), int(K),
+                                            _s(stream))
 
 
 def nvfp4_gemm_gateup_silu(X, M, wq_gate, ws_gate, gscale_gate, wq_up, ws_up, gscale_up, H, Nff, K,

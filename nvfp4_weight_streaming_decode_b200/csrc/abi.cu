@@ -50,6 +50,7 @@ extern "C" const char* nvfp4_status_string(int status)
     case NVFP4_ERR_CUDA: return "CUDA runtime error (see nvfp4_last_cuda_error)";
     case NVFP4_ERR_CAPTURE: return "first use of the device inside a stream capture";
     case NVFP4_ERR_DEVICE: return "a kernel's bounded wait gave up (see nvfp4_device_status)";
+    case NVFP4_ERR_SCRATCH: return "needs more scratch than the no-alloc entry point's static array holds";
     default: return "unknown status";
     }
 }

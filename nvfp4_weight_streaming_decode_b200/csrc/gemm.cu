@@ -635,6 +635,21 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
     return NVFP4_OK;
 }
 
+int gemm_launch_warps(const GemmArgs& a, DeviceState* ds, long long* warps)
+{
+    KernelInfo* k = nullptr;
+    int st = kernel_for(ds->device, a.kind, a.M, &k);
+    if (st != NVFP4_OK) return st;
+    const Geometry geo = geometry(a.N, a.K);
+    long long ctas = (long long)ds->sm_count * k->blocks_per_sm;
+    const long long need = (geo.units + kWarps - 1) / kWarps;
+    if (need < ctas) ctas = need;
+    *warps = ctas * kWarps;
+    return NVFP4_OK;
+}
+
+size_t gemm_workspace_floats_per_warp() { return 2 * (size_t)kSlotFloats; }
+
 int read_and_clear_device_status(int* status)
 {
     unsigned v = 0;

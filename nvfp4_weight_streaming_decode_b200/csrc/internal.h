@@ -56,6 +56,11 @@ int validate_gemm(const GemmArgs& a);
 // Resolve a kernel variant (attributes, occupancy) ahead of a stream capture.
 int prepare_kernel(DeviceState* ds, int kind, int M);
 
+// Warps the launch of `a` would use on this device (before any clamping to the
+// workspace), and the workspace floats each warp needs.
+int gemm_launch_warps(const GemmArgs& a, DeviceState* ds, long long* warps);
+size_t gemm_workspace_floats_per_warp();
+
 // Device-side status word (nonzero after a bounded wait gave up).
 int read_and_clear_device_status(int* status);
 
