@@ -44,6 +44,7 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--round-mode", default="chain", choices=["chain", "persistent"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="only warm-up and timed replays (for an ncu launch list)")
@@ -262,7 +263,7 @@ def gemm_sweep(dev, hbm_peak):
     G, D = abi.NVFP4_DESC_GEMM, abi.NVFP4_DESC_GATEUP_SILU
 
     def time_chain(descs, reps=10):
-        rnd = abi.Round(descs)
+        rnd = abi.Round(descs, abi.NVFP4_ROUND_CHAIN)
         with torch.cuda.stream(stream):
             for _ in range(3):
                 rnd.replay(8, stream)
@@ -369,8 +370,10 @@ def run_ours(args):
     w = synth.WORKLOADS[4]
 
     r = SyntheticRound.build(dev, layers=args.layers, hidden=w["hidden"], ffn=w["ffn"], vocab=w["vocab"])
-    rnd = abi.Round(r.descs)
-    nodes = rnd.nodes
+    mode = abi.NVFP4_ROUND_PERSISTENT if args.round_mode == "persistent" else abi.NVFP4_ROUND_CHAIN
+    rnd = abi.Round(r.descs, mode)
+    nodes = len(r.descs)          # GEMM nodes of the round (kernel launches in chain mode)
+    graph_nodes = rnd.nodes
     weight_bytes = r.weight_bytes
     io_bytes = round_io_bytes(r, M)
     stream = torch.cuda.Stream(device=dev)
@@ -435,16 +438,18 @@ def run_ours(args):
     e2e_value = world * weight_bytes * e2e_steps / e2e_s / 1e9
 
     # roofline of the decode GEMM kernel over the round: every node is a launch of it
-    per_launch_bytes = (weight_bytes + io_bytes) / nodes
-    per_launch_s = (elapsed_s / args.steps) / nodes
+    launches = graph_nodes            # kernel launches per round: 1 (persistent) or one per GEMM node (chain)
+    per_launch_bytes = (weight_bytes + io_bytes) / launches
+    per_launch_s = (elapsed_s / args.steps) / launches
     achieved = per_launch_bytes / per_launch_s / 1e9
     traffic_round = profiled_traffic()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak,
-                "traffic": (traffic_round / nodes) if traffic_round else None,
+                "traffic": (traffic_round / launches) if traffic_round else None,
                 "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
-                "kernel": "decode_gemm_kernel (all round nodes)"}
+                "kernel": ("round_kernel (persistent round, one launch per round)" if args.round_mode == "persistent"
+                           else "decode_gemm_kernel (one launch per round node)")}
 
     sweep = None
     if rank == 0 and not args.no_sweep:
@@ -464,7 +469,8 @@ def run_ours(args):
             "data": "synthetic (seeded random NVFP4 codes/scales, N(0,1) bf16 activations)",
             "config": {"workload": "round_64layers_head_m1to8", "width_M": M, "layers": args.layers,
                        "hidden": w["hidden"], "ffn": w["ffn"], "vocab": w["vocab"],
-                       "weight_bytes_per_round": weight_bytes, "graph_nodes": nodes,
+                       "weight_bytes_per_round": weight_bytes, "gemm_nodes": nodes,
+                       "graph_nodes": graph_nodes, "round_mode": args.round_mode,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (13.8 GB of weights per round)"},
             "round_ms": ms_per_step,
@@ -475,7 +481,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_host.numel() * 2,
                     "d2h_bytes_per_step": y_host.numel() * 4, "ms_per_step": e2e_s * 1e3 / e2e_steps},
-            "gpu_launches": nodes * args.steps,
+            "gpu_launches": graph_nodes * args.steps,
             "clocks": clk,
             "gemm_sweep": sweep,
         }

@@ -168,6 +168,24 @@ typedef struct {
  */
 NVFP4_API int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_round** out);
 
+/*
+ * nvfp4_round_create with a choice of how the round runs:
+ *   NVFP4_ROUND_CHAIN (what nvfp4_round_create uses): each width's graph holds
+ *     one kernel per node, linked by programmatic dependent launch (the chain
+ *     described above).  Results are bit-identical to direct calls.
+ *   NVFP4_ROUND_PERSISTENT: each width's graph holds one cooperative kernel
+ *     that runs every node in order on all SMs.  Each warp's weight stream
+ *     runs on from one node into the next, and a node's X is read only after
+ *     every CTA has finished the node before it (a counter per node, bounded
+ *     waits).  A fused gate/up node runs as one GEMM over both matrices
+ *     stacked into an FP32 buffer the round owns, then an elementwise
+ *     SiLU-multiply node; plain GEMM nodes keep the work split of a direct
+ *     call (bit-identical), fused ones agree with it within the GEMM bound.
+ *     At most 360 nodes per launch; longer rounds take several launches.
+ */
+enum { NVFP4_ROUND_PERSISTENT = 0, NVFP4_ROUND_CHAIN = 1 };
+NVFP4_API int nvfp4_round_create_ex(const nvfp4_gemm_desc* descs, int n, int mode, nvfp4_round** out);
+
 /* Number of kernel nodes in each of the round's graphs (host call). */
 NVFP4_API int nvfp4_round_nodes(const nvfp4_round* r, int* nodes);
 

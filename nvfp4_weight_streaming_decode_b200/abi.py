@@ -29,6 +29,8 @@ NVFP4_ERR_CUDA = -6
 NVFP4_ERR_CAPTURE = -7
 NVFP4_ERR_DEVICE = -8
 NVFP4_ERR_SCRATCH = -9
+NVFP4_ROUND_PERSISTENT = 0
+NVFP4_ROUND_CHAIN = 1
 NVFP4_DESC_GEMM = 0
 NVFP4_DESC_GATEUP_SILU = 1
 
@@ -51,6 +53,7 @@ _SIGNATURES = {
     "nvfp4_gemm_decode_noalloc": (_I, [_P, _I, _P, _P, _F, _P, _I64, _I64, _P]),
     "nvfp4_gemm_gateup_silu": (_I, [_P, _I, _P, _P, _F, _P, _P, _F, _P, _I64, _I64, _P]),
     "nvfp4_round_create": (_I, [ctypes.POINTER(Nvfp4GemmDesc), _I, ctypes.POINTER(_P)]),
+    "nvfp4_round_create_ex": (_I, [ctypes.POINTER(Nvfp4GemmDesc), _I, _I, ctypes.POINTER(_P)]),
     "nvfp4_round_nodes": (_I, [_P, ctypes.POINTER(_I)]),
     "nvfp4_round_replay": (_I, [_P, _I, _P]),
     "nvfp4_round_replay_host": (_I, [_P, _I, _P, _P, _SZ, _P, _P, _SZ, _P]),
@@ -148,6 +151,14 @@ def nvfp4_round_create(descs):
     arr = (Nvfp4GemmDesc * len(descs))(*descs)
     h = _P()
     st = load().nvfp4_round_create(arr, len(descs), ctypes.byref(h))
+    return st, h.value
+
+
+def nvfp4_round_create_ex(descs, mode):
+    """(status, handle) for a sequence of Nvfp4GemmDesc, with a round mode."""
+    arr = (Nvfp4GemmDesc * len(descs))(*descs)
+    h = _P()
+    st = load().nvfp4_round_create_ex(arr, len(descs), int(mode), ctypes.byref(h))
     return st, h.value
 
 
@@ -269,8 +280,11 @@ def unpack_debug(wq, ws, N, K, stream=None):
 class Round:
     """Owner of an nvfp4_round handle built from descriptors."""
 
-    def __init__(self, descs):
-        st, h = nvfp4_round_create(descs)
+    def __init__(self, descs, mode=None):
+        if mode is None:
+            st, h = nvfp4_round_create(descs)
+        else:
+            st, h = nvfp4_round_create_ex(descs, mode)
         check(st, "nvfp4_round_create")
         self.handle = h
         self._descs = list(descs)

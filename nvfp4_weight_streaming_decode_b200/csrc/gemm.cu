@@ -26,6 +26,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -222,21 +223,22 @@ __device__ __forceinline__ void load_partial(const float* src, float4 (&v)[NW * 
     for (int k = 0; k < NW * 2; ++k) v[k] = ld_cg_f4(src + 4 * k);
 }
 
-// End of a tile for this warp.  The warp has already stored its sums in its
-// partial slot.  A tile the warp covered alone goes straight to the
-// epilogue; otherwise the warp counts itself in, and the last contributor
-// adds every partial in warp order (glo..ghi, a fixed order, so the result
-// does not depend on who arrives last) and runs the epilogue.  Out of line,
-// so the streaming loop does not carry its registers.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// End of a tile for this warp, after it stored its sums in its partial slot.
+// A tile the warp covered alone goes straight to the epilogue.  Otherwise the
+// warp counts itself in, and the last contributor adds every partial in warp
+// order (glo..ghi, a fixed order, so the result does not depend on who arrives
+// last) and runs the epilogue.  Out of line, so the streaming loop does not
+// carry its registers.
 template <int M, int NW>
 __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane)
 {
     const long long U = o.units, TW = o.total_warps, KC = o.k_chunks;
     const long long ts = tile * KC, te = ts + KC;
     const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
-    float sum[NW][2][4];
     if (glo != ghi) {
-        __threadfence();
+        fence_acq_rel_gpu();
         __syncwarp();
         // Every warp below total_warps has a non-empty range, so the
         // contributors are exactly the warps glo..ghi.
@@ -244,16 +246,17 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         if (lane == 0) last = (atomicAdd(&o.counters[glo], 1u) == (unsigned)(ghi - glo)) ? 1u : 0u;
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) return;
-        __threadfence();
+        fence_acq_rel_gpu();
     }
     const int glo_slot = (range_begin(U, TW, glo) >= ts) ? 0 : 1;
+    float sum[NW][2][4];
 #pragma unroll
     for (int a = 0; a < NW; ++a)
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
-    constexpr int kBatch = NW == 1 ? 8 : 2;  // contributors whose loads are in flight together
+    constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together (more costs the callers spills)
     for (long long w0 = glo; w0 <= ghi; w0 += kBatch) {
         float4 v[kBatch][NW * 2];
 #pragma unroll
@@ -268,14 +271,12 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         for (int b = 0; b < kBatch; ++b) {
             if (w0 + b <= ghi) {
 #pragma unroll
-                for (int a = 0; a < NW; ++a)
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        sum[a][r][0] += v[b][a * 2 + r].x;
-                        sum[a][r][1] += v[b][a * 2 + r].y;
-                        sum[a][r][2] += v[b][a * 2 + r].z;
-                        sum[a][r][3] += v[b][a * 2 + r].w;
-                    }
+                for (int k = 0; k < NW * 2; ++k) {
+                    sum[k >> 1][k & 1][0] += v[b][k].x;
+                    sum[k >> 1][k & 1][1] += v[b][k].y;
+                    sum[k >> 1][k & 1][2] += v[b][k].z;
+                    sum[k >> 1][k & 1][3] += v[b][k].w;
+                }
             }
         }
     }
@@ -460,6 +461,328 @@ decode_gemm_kernel(const KParams p)
     }
 }
 
+// ------------------------------------------------------------------ persistent round
+//
+// The whole decode round as one cooperative launch: every warp walks the
+// nodes in order.  A GEMM node is done as a standalone launch would do it
+// (same stream-K partition); the fused gate/up node becomes one GEMM node
+// over both matrices stacked (gate rows, then up rows, into an FP32 buffer)
+// followed by an elementwise node H = bf16(silu(g) * u).  Each warp's
+// bulk-copy ring runs across node boundaries, so the next node's weights
+// (which depend on nothing) stream in while the current node drains.  Between
+// nodes the grid synchronises hierarchically: the warps of a CTA meet at a CTA
+// barrier, one thread per CTA counts the CTA in at the node's counter and
+// polls (bounded) until every CTA has, and a second CTA barrier releases the
+// warps.  All CTAs are co-resident (cooperative launch), so no wait depends on
+// a CTA that cannot run.
+
+enum { kNodeGemm = 0, kNodeSiluMul = 1 };
+
+struct RoundNode {
+    const uint8_t* wq[2];  // GEMM: planes A (units below split_units) and B
+    const uint8_t* ws[2];
+    const void* X;         // GEMM: bf16 [M][K];  SiLU-mul: FP32 [M][2*K] (g rows, then u rows)
+    void* out;             // GEMM: FP32 [M][N];  SiLU-mul: bf16 [M][N]
+    float gs[2];           // GEMM: global scale (gs[0]);  SiLU-mul: gate and up scales
+    int N, K, k_chunks, units, total_warps, split_units;
+    int kind;
+};
+
+// Passed whole as the kernel's parameter block (constant bank), so node
+// fields cost no registers; up to kMaxRoundNodes nodes per launch.
+constexpr int kMaxRoundNodes = 360;
+
+struct RoundParams {
+    float* partials;
+    unsigned* counters;
+    unsigned* arrive;  // per node: CTAs of the grid that finished it
+    int n_nodes;
+    int grid_ctas;
+    RoundNode nodes[kMaxRoundNodes];
+};
+
+constexpr int kRoundStages = 3;
+constexpr int kRoundUPS = 4;                        // GEMM units per stage
+constexpr int kRoundStageBytes = kRoundUPS * kUnitBytes;
+
+// Coherent 32-byte X load (X may have been written earlier in this launch).
+__device__ __forceinline__ void ld_x32_coherent(const void* p, bool pred, uint32_t (&x)[8])
+{
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.u32 q, %9, 0;\n"
+        " @q ld.global.v4.u32 {%0,%1,%2,%3}, [%8];\n"
+        " @q ld.global.v4.u32 {%4,%5,%6,%7}, [%8+16];\n}"
+        : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]), "+r"(x[7])
+        : "l"(p), "r"((uint32_t)pred)
+        : "memory");
+}
+
+// The bulk-copy side of a warp: which GEMM node and stage it issues next.
+// Lives in shared memory and is read and written by lane 0 only, so the
+// streaming loop carries none of it in registers.
+struct RoundIssuer {
+    int node, stage, n_stages, n_units;
+    int issued;  // stages issued so far (for the drain on the error path)
+    int u0;
+};
+
+// Move the issuer to the first GEMM node >= n where this warp has work (lane 0).
+__device__ __forceinline__ void issuer_seek(const RoundParams& rp, int gw, int n, RoundIssuer* is)
+{
+    for (; n < rp.n_nodes; ++n) {
+        const RoundNode& nd = rp.nodes[n];
+        if (nd.kind != kNodeGemm || gw >= nd.total_warps) continue;
+        const long long u0 = range_begin(nd.units, nd.total_warps, gw);
+        const long long u1 = range_begin(nd.units, nd.total_warps, gw + 1);
+        is->node = n;
+        is->stage = 0;
+        is->u0 = (int)u0;
+        is->n_units = (int)(u1 - u0);
+        is->n_stages = (is->n_units + kRoundUPS - 1) / kRoundUPS;
+        return;
+    }
+    is->node = rp.n_nodes;
+}
+
+// Issue the issuer's next stage into `slot` (lane 0 only).  A stage that
+// crosses from plane A to plane B is fetched with one copy from each.
+__device__ __forceinline__ void issuer_issue(const RoundParams& rp, int gw, uint32_t ring_s, uint32_t bar_s,
+                                             int slot, RoundIssuer* is)
+{
+    if (is->node >= rp.n_nodes) return;
+    const RoundNode& nd = rp.nodes[is->node];
+    const int ub = is->u0 + is->stage * kRoundUPS;
+    const int rem = is->n_units - is->stage * kRoundUPS;
+    const int cnt = rem < kRoundUPS ? rem : kRoundUPS;
+    const uint32_t dst = ring_s + slot * kRoundStageBytes;
+    const uint32_t bar = bar_s + 8 * slot;
+    const uint64_t pol = evict_first_policy();
+    mbar_expect_tx(bar, (uint32_t)(cnt * kUnitBytes));
+    const int split = nd.split_units;
+    const int na = ub >= split ? 0 : (split - ub < cnt ? split - ub : cnt);  // units from plane A
+    if (na > 0) {
+        bulk_load(dst, nd.wq[0] + (long long)ub * kUnitQ, na * kUnitQ, bar, pol);
+        bulk_load(dst + kRoundUPS * kUnitQ, nd.ws[0] + (long long)ub * kUnitS, na * kUnitS, bar, pol);
+    }
+    if (cnt > na) {
+        const long long b0 = (long long)(ub + na - split);
+        bulk_load(dst + na * kUnitQ, nd.wq[1] + b0 * kUnitQ, (cnt - na) * kUnitQ, bar, pol);
+        bulk_load(dst + kRoundUPS * kUnitQ + na * kUnitS, nd.ws[1] + b0 * kUnitS, (cnt - na) * kUnitS, bar, pol);
+    }
+    ++is->issued;
+    if (++is->stage == is->n_stages) issuer_seek(rp, gw, is->node + 1, is);
+}
+
+// This warp's stream-K range of one GEMM node.  Mirrors the standalone
+// kernel's loop; the ring (slot, parity) and the issuer carry over between
+// nodes.
+template <int M>
+__device__ __forceinline__ bool round_gemm(const RoundParams& rp, const RoundNode* cur, int gw, int lane,
+                                           uint8_t* ring, uint32_t ring_s, uint32_t bar_s, int& slot,
+                                           uint32_t& parity, RoundIssuer* is, int& consumed)
+{
+    const RoundNode& nd = *cur;
+    constexpr int UPS = kRoundUPS;
+    const int g = lane >> 2, t = lane & 3;
+    const long long TW = nd.total_warps, KC = nd.k_chunks;
+    const long long u0 = range_begin(nd.units, TW, gw), u1 = range_begin(nd.units, TW, gw + 1);
+    const int n_units = (int)(u1 - u0);
+    const int n_stages = (n_units + UPS - 1) / UPS;
+    float acc[1][2][4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[0][r][i] = 0.f;
+    long long tile = u0 / KC;
+    const long long first_tile = tile;
+    int chunk = (int)(u0 - tile * KC);
+    const int kc_last = (int)KC - 1;
+    const int K32 = nd.K;
+    const uint16_t* xp = static_cast<const uint16_t*>(nd.X) + (long long)(g < M ? g : 0) * nd.K + chunk * kChunkK + 16 * t;
+    int col = chunk * kChunkK + 16 * t;
+    const bool x_lane = g < M;
+    const uint32_t q_off = 16 * lane, s_off = 4 * lane;
+    uint32_t xf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    int i = 0;
+    for (int j = 0; j < n_stages; ++j) {
+        if (!warp_wait(bar_s + 8 * slot, parity)) return false;
+        ++consumed;
+        const uint8_t* stage = ring + slot * kRoundStageBytes;
+        if (n_units - i > UPS && kc_last - chunk >= UPS) {
+#pragma unroll
+            for (int v = 0; v < UPS; ++v) {
+                ld_x32_coherent(xp + v * kChunkK, x_lane, xf);
+                mma_unit(stage + v * kUnitQ + q_off, stage + UPS * kUnitQ + v * kUnitS + s_off, xf, acc[0]);
+            }
+            i += UPS;
+            chunk += UPS;
+            col += UPS * kChunkK;
+            xp += UPS * kChunkK;
+        } else {
+#pragma unroll 1
+            for (int v = 0; v < UPS; ++v) {
+                if (i < n_units) {
+                    uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                    ld_x32_coherent(xp, x_lane && col < K32, xw);
+                    mma_unit(stage + v * kUnitQ + q_off, stage + UPS * kUnitQ + v * kUnitS + s_off, xw, acc[0]);
+                    ++i;
+                    const bool tile_end = chunk == kc_last;
+                    if (tile_end || i == n_units) {
+                        const int slot_id = (tile == first_tile) ? 0 : 1;
+                        float* dst = rp.partials + ((size_t)gw * 2 + slot_id) * kSlotFloats + lane * 8;
+#pragma unroll
+                        for (int r = 0; r < 2; ++r)
+                            reinterpret_cast<float4*>(dst)[r] =
+                                make_float4(acc[0][r][0], acc[0][r][1], acc[0][r][2], acc[0][r][3]);
+                        // Node fields for the epilogue come from shared memory here, so the
+                        // streaming loop does not keep them in registers.
+                        volatile const RoundNode* vn = cur;
+                        OutArgs o;
+                        o.out = vn->out;
+                        o.partials = rp.partials;
+                        o.counters = rp.counters;
+                        o.N = vn->N;
+                        o.units = vn->units;
+                        o.total_warps = vn->total_warps;
+                        o.k_chunks = vn->k_chunks;
+                        o.gs0 = vn->gs[0];
+                        o.gs1 = vn->gs[1];
+                        tile_done<M, 1>(o, tile, lane);
+#pragma unroll
+                        for (int r = 0; r < 2; ++r)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) acc[0][r][k] = 0.f;
+                    }
+                    if (tile_end) {
+                        ++tile;
+                        chunk = 0;
+                        col = 16 * t;
+                        xp -= kc_last * kChunkK;
+                    } else {
+                        ++chunk;
+                        col += kChunkK;
+                        xp += kChunkK;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) issuer_issue(rp, gw, ring_s, bar_s, slot, is);
+        if (++slot == kRoundStages) {
+            slot = 0;
+            parity ^= 1u;
+        }
+    }
+    return true;
+}
+
+// H[m][n] = bf16(silu(g) * u) with g = X[m][n] * gs[0], u = X[m][P + n] * gs[1]
+// (P = nd.K; X holds the stacked GEMM's acc * 2^8, so each product is the
+// single rounding the fused kernel's epilogue makes).
+template <int M>
+__device__ __forceinline__ void round_silu_mul(const RoundNode& nd, int gtid, int nthreads)
+{
+    const float* gu = static_cast<const float*>(nd.X);
+    __nv_bfloat16* H = static_cast<__nv_bfloat16*>(nd.out);
+    const int N = nd.N, P = nd.K;
+    for (int e = gtid; e < M * N; e += nthreads) {
+        const int m = e / N, n = e - m * N;
+        float gv, uv;
+        asm volatile("ld.global.f32 %0, [%1];" : "=f"(gv) : "l"(gu + (long long)m * 2 * P + n) : "memory");
+        asm volatile("ld.global.f32 %0, [%1];" : "=f"(uv) : "l"(gu + (long long)m * 2 * P + P + n) : "memory");
+        gv *= nd.gs[0];
+        uv *= nd.gs[1];
+        H[(long long)m * N + n] = __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
+    }
+}
+
+// Bounded wait until `*ctr >= target` (one thread, acquire semantics).
+__device__ __forceinline__ bool wait_count_thread(const unsigned* ctr, unsigned target)
+{
+    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) return true;
+        __nanosleep(32);
+    }
+    return false;
+}
+
+template <int M>
+__global__ void __launch_bounds__(kWarps * 32, 1) round_kernel(const RoundParams rp)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ RoundIssuer issuers[kWarps];
+    __shared__ RoundNode cur_node;  // the node being worked on (copied by thread 0 at each node start)
+    __shared__ int cta_ok;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int gw = blockIdx.x * kWarps + warp;
+
+    uint8_t* ring = smem + warp * (kRoundStages * kRoundStageBytes);
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t bar_s = smem_addr(smem + kWarps * kRoundStages * kRoundStageBytes) + warp * kRoundStages * 8;
+    RoundIssuer* is = issuers + warp;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kRoundStages; ++s) mbar_init(bar_s + 8 * s);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        is->issued = 0;
+        issuer_seek(rp, gw, 0, is);
+        for (int s = 0; s < kRoundStages; ++s) issuer_issue(rp, gw, ring_s, bar_s, s, is);
+    }
+    if (threadIdx.x == 0) {
+        cta_ok = 1;
+        cur_node = rp.nodes[0];
+    }
+    __syncthreads();
+
+    int slot = 0, consumed = 0;
+    uint32_t parity = 0;
+    bool ok = true;
+    for (int c = 0; c < rp.n_nodes; ++c) {
+        if (cur_node.kind == kNodeGemm) {
+            if (gw < cur_node.total_warps)
+                ok = round_gemm<M>(rp, &cur_node, gw, lane, ring, ring_s, bar_s, slot, parity, is, consumed);
+        } else {
+            round_silu_mul<M>(cur_node, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
+        }
+        if (!ok && lane == 0) atomicAnd(&cta_ok, 0);
+        // Grid barrier: this CTA's warps meet, one thread counts the CTA in and
+        // waits for all CTAs, then releases the CTA.
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(rp.arrive + c, 1u);
+            if (cta_ok && !wait_count_thread(rp.arrive + c, (unsigned)rp.grid_ctas)) cta_ok = 0;
+            __threadfence();
+            if (c + 1 < rp.n_nodes) cur_node = rp.nodes[c + 1];
+        }
+        __syncthreads();
+        if (!cta_ok) break;
+    }
+    if (threadIdx.x == 0 && cta_ok) {
+        // The last CTA to get here resets the counters for the next launch.
+        const unsigned done = atomicAdd(rp.arrive + rp.n_nodes, 1u);
+        if (done == (unsigned)rp.grid_ctas - 1) {
+            for (int k = 0; k <= rp.n_nodes; ++k) rp.arrive[k] = 0u;
+        }
+    }
+    if (!cta_ok) {
+        // Give up: flag it, then wait (bounded) for this warp's copies still in flight.
+        if (threadIdx.x == 0) atomicOr(&g_device_status, 2u);
+        __syncwarp();
+        const int issued = is->issued;
+        for (int s = consumed; s < issued; ++s) {
+            warp_wait(bar_s + 8 * slot, parity);
+            if (++slot == kRoundStages) {
+                slot = 0;
+                parity ^= 1u;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 namespace {
@@ -632,6 +955,136 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
     cfg.numAttrs = pdl ? 1 : 0;
     void* args[] = {&p};
     NVFP4_CUDA_TRY(cudaLaunchKernelExC(&cfg, k->fn, args));
+    return NVFP4_OK;
+}
+
+namespace {
+
+template <int M>
+void* round_kernel_fn()
+{
+    return (void*)round_kernel<M>;
+}
+
+void* round_kernel_for(int M)
+{
+    switch (M) {
+    case 1: return round_kernel_fn<1>();
+    case 2: return round_kernel_fn<2>();
+    case 3: return round_kernel_fn<3>();
+    case 4: return round_kernel_fn<4>();
+    case 5: return round_kernel_fn<5>();
+    case 6: return round_kernel_fn<6>();
+    case 7: return round_kernel_fn<7>();
+    default: return round_kernel_fn<8>();
+    }
+}
+
+constexpr size_t kRoundSmem = (size_t)kWarps * kRoundStages * (kRoundStageBytes + 8);
+
+}  // namespace
+
+int round_persistent_params_size() { return (int)sizeof(RoundParams); }
+int round_persistent_max_nodes() { return kMaxRoundNodes; }
+
+size_t round_persistent_temp_floats(const GemmArgs* nodes, int n)
+{
+    size_t need = 0;
+    for (int i = 0; i < n; ++i)
+        if (nodes[i].kind == 1) {
+            const size_t p = (size_t)geometry(nodes[i].N, nodes[i].K).n_tiles * kTileN;
+            if (2 * p * kMaxM > need) need = 2 * p * kMaxM;
+        }
+    return need;
+}
+
+// Expands descriptors into round nodes; a fused gate/up descriptor becomes a
+// stacked GEMM node (into `temp`) plus a SiLU-multiply node.  Returns the
+// node count in *count, or NVFP4_ERR_ARG if more than kMaxRoundNodes result.
+int round_persistent_build(const GemmArgs* nodes, int n, DeviceState* ds, float* temp, void* params_host,
+                           int* count)
+{
+    RoundParams* rp = static_cast<RoundParams*>(params_host);
+    memset(rp, 0, sizeof(RoundParams));
+    int k = 0;
+    for (int i = 0; i < n; ++i) {
+        const GemmArgs& a = nodes[i];
+        const Geometry geo = geometry(a.N, a.K);
+        const int fused = a.kind == 1;
+        if (k + 1 + fused > kMaxRoundNodes) return NVFP4_ERR_ARG;
+        GemmArgs g = a;
+        g.kind = 0;
+        long long rows = a.N;
+        if (fused) rows = 2 * geo.n_tiles * (long long)kTileN;  // gate rows, then up rows (tile-padded)
+        g.N = rows;
+        long long warps = 0;
+        int st = gemm_launch_warps(g, ds, &warps);
+        if (st != NVFP4_OK) return st;
+        const long long units = fused ? 2 * geo.units : geo.units;
+        if (units > 0x7fffffffLL || rows > 0x7fffffffLL || a.K > 0x7fffffffLL) return NVFP4_ERR_SHAPE;
+        RoundNode& r = rp->nodes[k++];
+        r.kind = kNodeGemm;
+        r.wq[0] = a.wq[0];
+        r.ws[0] = a.ws[0];
+        r.wq[1] = fused ? a.wq[1] : a.wq[0];
+        r.ws[1] = fused ? a.ws[1] : a.ws[0];
+        r.gs[0] = fused ? 1.0f : a.gscale[0];  // a stacked gate/up node leaves the scales to its SiLU node
+        r.gs[1] = r.gs[0];
+        r.X = a.X;
+        r.out = fused ? (void*)temp : a.out;
+        r.N = (int)rows;
+        r.K = (int)a.K;
+        r.k_chunks = (int)geo.k_chunks;
+        r.units = (int)units;
+        r.total_warps = (int)(warps < units ? warps : units);  // a standalone launch's partition
+        r.split_units = (int)geo.units;
+        if (fused) {
+            RoundNode& h = rp->nodes[k++];
+            memset(&h, 0, sizeof h);
+            h.kind = kNodeSiluMul;
+            h.X = temp;
+            h.out = a.out;
+            h.N = (int)a.N;
+            h.K = (int)(geo.n_tiles * kTileN);
+            h.gs[0] = a.gscale[0];
+            h.gs[1] = a.gscale[1];
+        }
+    }
+    rp->n_nodes = k;
+    rp->partials = ds->partials;
+    rp->counters = ds->counters;
+    *count = k;
+    return NVFP4_OK;
+}
+
+int round_persistent_prepare(DeviceState* ds, int M, int* grid)
+{
+    void* fn = round_kernel_for(M);
+    NVFP4_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRoundSmem));
+    int nb = 0;
+    NVFP4_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kWarps * 32, kRoundSmem));
+    if (nb < 1) return NVFP4_ERR_CUDA;
+    *grid = ds->sm_count;  // one CTA per SM, all co-resident
+    return NVFP4_OK;
+}
+
+int round_persistent_launch(void* params_host, unsigned* d_arrive, int M, int grid, cudaStream_t stream)
+{
+    RoundParams* rp = static_cast<RoundParams*>(params_host);
+    rp->arrive = d_arrive;
+    rp->grid_ctas = grid;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = kRoundSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {rp};
+    NVFP4_CUDA_TRY(cudaLaunchKernelExC(&cfg, round_kernel_for(M), args));
     return NVFP4_OK;
 }
 

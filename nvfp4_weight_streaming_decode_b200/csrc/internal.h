@@ -61,6 +61,17 @@ int prepare_kernel(DeviceState* ds, int kind, int M);
 int gemm_launch_warps(const GemmArgs& a, DeviceState* ds, long long* warps);
 size_t gemm_workspace_floats_per_warp();
 
+// The persistent round: per-width preparation and the cooperative launch.
+// The node table travels as the kernel's parameter block (host buffer of
+// round_persistent_params_size() bytes, at most 300 nodes per launch).
+int round_persistent_params_size();
+int round_persistent_max_nodes();
+size_t round_persistent_temp_floats(const GemmArgs* nodes, int n);
+int round_persistent_build(const GemmArgs* nodes, int n, DeviceState* ds, float* temp, void* params_host,
+                           int* count);
+int round_persistent_prepare(DeviceState* ds, int M, int* grid);
+int round_persistent_launch(void* params_host, unsigned* d_arrive, int M, int grid, cudaStream_t stream);
+
 // Device-side status word (nonzero after a bounded wait gave up).
 int read_and_clear_device_status(int* status);
 

@@ -15,6 +15,11 @@
 struct nvfp4_round {
     int device;
     int n;
+    int mode;                 // NVFP4_ROUND_PERSISTENT or NVFP4_ROUND_CHAIN
+    int n_chunks;             // persistent mode: launches per round (node tables of at most 360 nodes)
+    void** params;            // persistent mode: host copies of the kernel parameter blocks, per chunk
+    unsigned** d_arrive;      // persistent mode: per-chunk arrival counters (nodes + 1)
+    float* d_temp;            // persistent mode: FP32 gate/up results of a fused node
     nvfp4_gemm_desc* descs;
     cudaStream_t stream;
     cudaGraph_t graphs[nvfp4::kMaxM];
@@ -50,6 +55,13 @@ void release(nvfp4_round* r)
         if (r->graphs[i]) cudaGraphDestroy(r->graphs[i]);
     }
     if (r->stream) cudaStreamDestroy(r->stream);
+    for (int c = 0; c < r->n_chunks; ++c) {
+        if (r->params) free(r->params[c]);
+        if (r->d_arrive && r->d_arrive[c]) cudaFree(r->d_arrive[c]);
+    }
+    free(r->params);
+    free(r->d_arrive);
+    if (r->d_temp) cudaFree(r->d_temp);
     free(r->descs);
     free(r);
 }
@@ -58,8 +70,14 @@ void release(nvfp4_round* r)
 
 extern "C" int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_round** out)
 {
+    return nvfp4_round_create_ex(descs, n, NVFP4_ROUND_CHAIN, out);
+}
+
+extern "C" int nvfp4_round_create_ex(const nvfp4_gemm_desc* descs, int n, int mode, nvfp4_round** out)
+{
     using namespace nvfp4;
     if (!descs || !out || n < 1) return NVFP4_ERR_ARG;
+    if (mode != NVFP4_ROUND_PERSISTENT && mode != NVFP4_ROUND_CHAIN) return NVFP4_ERR_ARG;
     *out = nullptr;
     for (int i = 0; i < n; ++i) {
         const GemmArgs a = args_of(descs[i], kMaxM);
@@ -75,6 +93,7 @@ extern "C" int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_rou
     }
     memcpy(r->descs, descs, sizeof(nvfp4_gemm_desc) * (size_t)n);
     r->n = n;
+    r->mode = mode;
     cudaError_t e = cudaGetDevice(&r->device);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r->stream, cudaStreamNonBlocking);
     if (e != cudaSuccess) {
@@ -86,6 +105,45 @@ extern "C" int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_rou
     // Resolve every kernel (attributes, occupancy) outside the capture.
     for (int M = 1; st == NVFP4_OK && M <= kMaxM; ++M)
         for (int k = 0; st == NVFP4_OK && k < 2; ++k) st = prepare_kernel(ds, k, M);
+    int grid = 0;
+    if (st == NVFP4_OK && mode == NVFP4_ROUND_PERSISTENT) {
+        for (int M = 1; st == NVFP4_OK && M <= kMaxM; ++M) st = round_persistent_prepare(ds, M, &grid);
+        GemmArgs* args = (GemmArgs*)malloc(sizeof(GemmArgs) * (size_t)n);
+        if (!args) st = NVFP4_ERR_ARG;
+        for (int i = 0; st == NVFP4_OK && i < n; ++i) args[i] = args_of(r->descs[i], kMaxM);
+        const size_t temp_floats = st == NVFP4_OK ? round_persistent_temp_floats(args, n) : 0;
+        if (st == NVFP4_OK && temp_floats) {
+            e = cudaMalloc(&r->d_temp, temp_floats * sizeof(float));
+            if (e != cudaSuccess) st = fail_cuda(e);
+        }
+        // Chunks of descriptors whose expanded node tables fit one launch's parameter block.
+        const int cap = round_persistent_max_nodes();
+        r->params = (void**)calloc((size_t)n, sizeof(void*));
+        r->d_arrive = (unsigned**)calloc((size_t)n, sizeof(unsigned*));
+        if (!r->params || !r->d_arrive) st = NVFP4_ERR_ARG;
+        for (int i0 = 0; st == NVFP4_OK && i0 < n;) {
+            int i1 = i0, nodes = 0;
+            while (i1 < n && nodes + 1 + (args[i1].kind == 1) <= cap) nodes += 1 + (args[i1++].kind == 1);
+            const int c = r->n_chunks++;
+            r->params[c] = malloc((size_t)round_persistent_params_size());
+            if (!r->params[c]) {
+                st = NVFP4_ERR_ARG;
+                break;
+            }
+            int count = 0;
+            st = round_persistent_build(args + i0, i1 - i0, ds, r->d_temp, r->params[c], &count);
+            if (st != NVFP4_OK) break;
+            e = cudaMalloc(&r->d_arrive[c], sizeof(unsigned) * (size_t)(count + 1));
+            if (e == cudaSuccess) e = cudaMemset(r->d_arrive[c], 0, sizeof(unsigned) * (size_t)(count + 1));
+            if (e != cudaSuccess) st = fail_cuda(e);
+            i0 = i1;
+        }
+        if (st == NVFP4_OK) {
+            e = cudaDeviceSynchronize();
+            if (e != cudaSuccess) st = fail_cuda(e);
+        }
+        free(args);
+    }
     for (int M = 1; st == NVFP4_OK && M <= kMaxM; ++M) {
         e = cudaStreamBeginCapture(r->stream, cudaStreamCaptureModeThreadLocal);
         if (e != cudaSuccess) {
@@ -93,8 +151,12 @@ extern "C" int nvfp4_round_create(const nvfp4_gemm_desc* descs, int n, nvfp4_rou
             break;
         }
         int lst = NVFP4_OK;
-        for (int i = 0; i < n && lst == NVFP4_OK; ++i)
-            lst = launch_gemm(args_of(r->descs[i], M), r->stream, i > 0, ds);
+        if (mode == NVFP4_ROUND_PERSISTENT)
+            for (int c = 0; c < r->n_chunks && lst == NVFP4_OK; ++c)
+                lst = round_persistent_launch(r->params[c], r->d_arrive[c], M, grid, r->stream);
+        else
+            for (int i = 0; i < n && lst == NVFP4_OK; ++i)
+                lst = launch_gemm(args_of(r->descs[i], M), r->stream, i > 0, ds);
         cudaGraph_t graph = nullptr;
         e = cudaStreamEndCapture(r->stream, &graph);
         r->graphs[M - 1] = graph;
