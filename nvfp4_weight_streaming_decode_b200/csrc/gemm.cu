@@ -229,24 +229,33 @@ __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_re
 // A tile the warp covered alone goes straight to the epilogue.  Otherwise the
 // warp counts itself in, and the last contributor adds every partial in warp
 // order (glo..ghi, a fixed order, so the result does not depend on who arrives
-// last) and runs the epilogue.  Out of line, so the streaming loop does not
-// carry its registers.
+// last) and runs the epilogue.  When the finishing warp's bulk-copy ring is
+// idle (its range is done; gather_smem != 0) and the partials fit, they are
+// gathered into it with one bulk copy per contributor, all in flight at once;
+// otherwise they are loaded a few contributors at a time.  Out of line, so
+// the streaming loop does not carry its registers.
 template <int M, int NW>
-__device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane)
+__device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane, uint32_t gather_smem,
+                                       uint32_t gather_bytes, uint32_t gather_bar)
 {
     const long long U = o.units, TW = o.total_warps, KC = o.k_chunks;
     const long long ts = tile * KC, te = ts + KC;
     const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
     if (glo != ghi) {
-        fence_acq_rel_gpu();
+        // The lanes' partial stores are ordered before lane 0's release by the
+        // warp barrier; the acquire side of the same atomic orders the last
+        // contributor's reads of the other partials after it.
         __syncwarp();
         // Every warp below total_warps has a non-empty range, so the
         // contributors are exactly the warps glo..ghi.
         unsigned last = 0;
-        if (lane == 0) last = (atomicAdd(&o.counters[glo], 1u) == (unsigned)(ghi - glo)) ? 1u : 0u;
+        if (lane == 0) {
+            unsigned old;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(o.counters + glo) : "memory");
+            last = (old == (unsigned)(ghi - glo)) ? 1u : 0u;
+        }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) return;
-        fence_acq_rel_gpu();
     }
     const int glo_slot = (range_begin(U, TW, glo) >= ts) ? 0 : 1;
     float sum[NW][2][4];
@@ -256,26 +265,67 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
-    constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together (more costs the callers spills)
-    for (long long w0 = glo; w0 <= ghi; w0 += kBatch) {
-        float4 v[kBatch][NW * 2];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const long long w = w0 + b;
-            if (w <= ghi) {
-                const int ws = (w == glo) ? glo_slot : 0;
-                load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
-            }
+    const int C = (int)(ghi - glo + 1);
+    constexpr uint32_t kPartBytes = NW * 1024;  // the used part of a slot: 32 lanes x NW x 8 floats
+    bool gathered = false;
+    if (gather_smem != 0 && (uint32_t)C * kPartBytes <= gather_bytes) {
+        // order this warp's earlier reads of the ring, and the partials it
+        // acquired, before the bulk copies (async proxy)
+        asm volatile("fence.proxy.async;" ::: "memory");
+        if (lane == 0) mbar_expect_tx(gather_bar, (uint32_t)C * kPartBytes);
+        __syncwarp();
+        for (int c = lane; c < C; c += 32) {
+            const long long w = glo + c;
+            const int ws = (w == glo) ? glo_slot : 0;
+            const uint64_t pol = evict_first_policy();
+            bulk_load(gather_smem + c * kPartBytes, o.partials + ((size_t)w * 2 + ws) * kSlotFloats, kPartBytes,
+                      gather_bar, pol);
         }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            if (w0 + b <= ghi) {
+        // used once per warp and kernel, so the phase is always 0
+        gathered = warp_wait(gather_bar, 0u);
+        if (gathered) {
+            for (int c = 0; c < C; ++c) {
+                const uint32_t src = gather_smem + c * kPartBytes + lane * (NW * 32);
 #pragma unroll
                 for (int k = 0; k < NW * 2; ++k) {
-                    sum[k >> 1][k & 1][0] += v[b][k].x;
-                    sum[k >> 1][k & 1][1] += v[b][k].y;
-                    sum[k >> 1][k & 1][2] += v[b][k].z;
-                    sum[k >> 1][k & 1][3] += v[b][k].w;
+                    float4 x;
+                    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                 : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                                 : "r"(src + 16 * k));
+                    sum[k >> 1][k & 1][0] += x.x;
+                    sum[k >> 1][k & 1][1] += x.y;
+                    sum[k >> 1][k & 1][2] += x.z;
+                    sum[k >> 1][k & 1][3] += x.w;
+                }
+            }
+        } else {
+            // give up on the gather (flagged); wait once more, bounded, for the copies
+            if (lane == 0) atomicOr(&g_device_status, 4u);
+            warp_wait(gather_bar, 0u);
+        }
+    }
+    if (!gathered) {
+        constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together (more costs the callers spills)
+        for (long long w0 = glo; w0 <= ghi; w0 += kBatch) {
+            float4 v[kBatch][NW * 2];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const long long w = w0 + b;
+                if (w <= ghi) {
+                    const int ws = (w == glo) ? glo_slot : 0;
+                    load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                if (w0 + b <= ghi) {
+#pragma unroll
+                    for (int k = 0; k < NW * 2; ++k) {
+                        sum[k >> 1][k & 1][0] += v[b][k].x;
+                        sum[k >> 1][k & 1][1] += v[b][k].y;
+                        sum[k >> 1][k & 1][2] += v[b][k].z;
+                        sum[k >> 1][k & 1][3] += v[b][k].w;
+                    }
                 }
             }
         }
@@ -311,10 +361,13 @@ decode_gemm_kernel(const KParams p)
     uint8_t* ring = smem + warp * (STAGES * kStage);
     const uint32_t ring_s = smem_addr(ring);
     const uint32_t bar_s = smem_addr(smem + kWarps * STAGES * kStage) + warp * STAGES * 8;
+    // one more mbarrier per warp, for gathering partial sums into the idle ring
+    const uint32_t gather_bar = smem_addr(smem + kWarps * STAGES * (kStage + 8)) + warp * 8;
 
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) mbar_init(bar_s + 8 * s);
+        mbar_init(gather_bar);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncwarp();
@@ -429,7 +482,9 @@ decode_gemm_kernel(const KParams p)
                     o.k_chunks = p.k_chunks;
                     o.gs0 = p.gs[0];
                     o.gs1 = p.gs[1];
-                    tile_done<M, NW>(o, tile, lane);
+                    // At the end of the range every stage has been consumed and no copy is
+                    // in flight, so the ring can take the partial sums of a combine.
+                    tile_done<M, NW>(o, tile, lane, i == n_units ? ring_s : 0u, STAGES * kStage, gather_bar);
 #pragma unroll
                     for (int a = 0; a < NW; ++a)
 #pragma unroll
@@ -647,7 +702,7 @@ __device__ __forceinline__ bool round_gemm(const RoundParams& rp, const RoundNod
                         o.k_chunks = vn->k_chunks;
                         o.gs0 = vn->gs[0];
                         o.gs1 = vn->gs[1];
-                        tile_done<M, 1>(o, tile, lane);
+                        tile_done<M, 1>(o, tile, lane, 0u, 0u, 0u);
 #pragma unroll
                         for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -795,7 +850,7 @@ struct KernelOf {
     static constexpr int stages = NW == 1 ? kStagesPlain : kStagesFused;
     static constexpr int ups = NW == 1 ? kUnitsPerStagePlain : kUnitsPerStageFused;
     static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages, ups>; }
-    static size_t smem() { return (size_t)kWarps * stages * (NW * ups * kUnitBytes + 8); }
+    static size_t smem() { return (size_t)kWarps * stages * (NW * ups * kUnitBytes + 8) + kWarps * 8; }
 };
 
 struct KernelInfo {
