@@ -229,11 +229,14 @@ __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_re
 // A tile the warp covered alone goes straight to the epilogue.  Otherwise the
 // warp counts itself in, and the last contributor adds every partial in warp
 // order (glo..ghi, a fixed order, so the result does not depend on who arrives
-// last) and runs the epilogue.  When the finishing warp's bulk-copy ring is
-// idle (its range is done; gather_smem != 0) and the partials fit, they are
-// gathered into it with one bulk copy per contributor, all in flight at once;
-// otherwise they are loaded a few contributors at a time.  Out of line, so
-// the streaming loop does not carry its registers.
+// last) and runs the epilogue.  A warp that finds every other contributor
+// already counted in is the last one without counting itself in, which saves
+// the release and the atomic's round trip on the path that ends the kernel.
+// When the finishing warp's bulk-copy ring is idle (its range is done;
+// gather_smem != 0), the first contributors' partials are gathered into it
+// with one bulk copy each, all in flight at once, and the rest are loaded
+// into registers a few at a time, the first few while the copies are in
+// flight.  Out of line, so the streaming loop does not carry its registers.
 template <int M, int NW>
 __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane, uint32_t gather_smem,
                                        uint32_t gather_bytes, uint32_t gather_bar)
@@ -243,16 +246,23 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
     const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
     if (glo != ghi) {
         // The lanes' partial stores are ordered before lane 0's release by the
-        // warp barrier; the acquire side of the same atomic orders the last
-        // contributor's reads of the other partials after it.
+        // warp barrier; the acquire side (of the load or of the atomic) orders
+        // the last contributor's reads of the other partials after theirs.
         __syncwarp();
         // Every warp below total_warps has a non-empty range, so the
         // contributors are exactly the warps glo..ghi.
         unsigned last = 0;
         if (lane == 0) {
-            unsigned old;
-            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(o.counters + glo) : "memory");
-            last = (old == (unsigned)(ghi - glo)) ? 1u : 0u;
+            const unsigned others = (unsigned)(ghi - glo);
+            unsigned seen;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(o.counters + glo) : "memory");
+            if (seen == others) {
+                last = 1u;
+            } else {
+                unsigned old;
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(o.counters + glo) : "memory");
+                last = (old == others) ? 1u : 0u;
+            }
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) return;
@@ -267,66 +277,86 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
             for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
     const int C = (int)(ghi - glo + 1);
     constexpr uint32_t kPartBytes = NW * 1024;  // the used part of a slot: 32 lanes x NW x 8 floats
-    bool gathered = false;
-    if (gather_smem != 0 && (uint32_t)C * kPartBytes <= gather_bytes) {
+    // contributors 0..nb-1 through the ring, nb..C-1 through registers
+    int nb = gather_smem != 0 ? (int)(gather_bytes / kPartBytes) : 0;
+    if (nb > C) nb = C;
+    if (nb > 0) {
         // order this warp's earlier reads of the ring, and the partials it
         // acquired, before the bulk copies (async proxy)
         asm volatile("fence.proxy.async;" ::: "memory");
-        if (lane == 0) mbar_expect_tx(gather_bar, (uint32_t)C * kPartBytes);
+        if (lane == 0) mbar_expect_tx(gather_bar, (uint32_t)nb * kPartBytes);
         __syncwarp();
-        for (int c = lane; c < C; c += 32) {
+        for (int c = lane; c < nb; c += 32) {
             const long long w = glo + c;
             const int ws = (w == glo) ? glo_slot : 0;
             const uint64_t pol = evict_first_policy();
             bulk_load(gather_smem + c * kPartBytes, o.partials + ((size_t)w * 2 + ws) * kSlotFloats, kPartBytes,
                       gather_bar, pol);
         }
-        // used once per warp and kernel, so the phase is always 0
-        gathered = warp_wait(gather_bar, 0u);
-        if (gathered) {
-            for (int c = 0; c < C; ++c) {
-                const uint32_t src = gather_smem + c * kPartBytes + lane * (NW * 32);
+    }
+    constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together (more costs the callers spills)
+    float4 v[kBatch][NW * 2];
+    long long w0 = glo + nb;
 #pragma unroll
-                for (int k = 0; k < NW * 2; ++k) {
-                    float4 x;
-                    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                                 : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
-                                 : "r"(src + 16 * k));
-                    sum[k >> 1][k & 1][0] += x.x;
-                    sum[k >> 1][k & 1][1] += x.y;
-                    sum[k >> 1][k & 1][2] += x.z;
-                    sum[k >> 1][k & 1][3] += x.w;
-                }
-            }
-        } else {
-            // give up on the gather (flagged); wait once more, bounded, for the copies
+    for (int b = 0; b < kBatch; ++b) {
+        const long long w = w0 + b;
+        if (w <= ghi) {
+            const int ws = (w == glo) ? glo_slot : 0;
+            load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
+        }
+    }
+    if (nb > 0) {
+        // used once per warp and kernel, so the phase is always 0
+        const bool gathered = warp_wait(gather_bar, 0u);
+        if (!gathered) {
+            // flag it, wait once more (bounded) for the copies, and read these partials from global memory
             if (lane == 0) atomicOr(&g_device_status, 4u);
             warp_wait(gather_bar, 0u);
         }
-    }
-    if (!gathered) {
-        constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together (more costs the callers spills)
-        for (long long w0 = glo; w0 <= ghi; w0 += kBatch) {
-            float4 v[kBatch][NW * 2];
+        for (int c = 0; c < nb; ++c) {
+            float4 x[NW * 2];
+            if (gathered) {
+                const uint32_t src = gather_smem + c * kPartBytes + lane * (NW * 32);
 #pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-                const long long w = w0 + b;
-                if (w <= ghi) {
-                    const int ws = (w == glo) ? glo_slot : 0;
-                    load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
-                }
+                for (int k = 0; k < NW * 2; ++k)
+                    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                 : "=f"(x[k].x), "=f"(x[k].y), "=f"(x[k].z), "=f"(x[k].w)
+                                 : "r"(src + 16 * k));
+            } else {
+                const long long w = glo + c;
+                const int ws = (w == glo) ? glo_slot : 0;
+                load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), x);
             }
 #pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-                if (w0 + b <= ghi) {
+            for (int k = 0; k < NW * 2; ++k) {
+                sum[k >> 1][k & 1][0] += x[k].x;
+                sum[k >> 1][k & 1][1] += x[k].y;
+                sum[k >> 1][k & 1][2] += x[k].z;
+                sum[k >> 1][k & 1][3] += x[k].w;
+            }
+        }
+    }
+    for (;;) {
 #pragma unroll
-                    for (int k = 0; k < NW * 2; ++k) {
-                        sum[k >> 1][k & 1][0] += v[b][k].x;
-                        sum[k >> 1][k & 1][1] += v[b][k].y;
-                        sum[k >> 1][k & 1][2] += v[b][k].z;
-                        sum[k >> 1][k & 1][3] += v[b][k].w;
-                    }
+        for (int b = 0; b < kBatch; ++b) {
+            if (w0 + b <= ghi) {
+#pragma unroll
+                for (int k = 0; k < NW * 2; ++k) {
+                    sum[k >> 1][k & 1][0] += v[b][k].x;
+                    sum[k >> 1][k & 1][1] += v[b][k].y;
+                    sum[k >> 1][k & 1][2] += v[b][k].z;
+                    sum[k >> 1][k & 1][3] += v[b][k].w;
                 }
+            }
+        }
+        w0 += kBatch;
+        if (w0 > ghi) break;
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const long long w = w0 + b;
+            if (w <= ghi) {
+                const int ws = (w == glo) ? glo_slot : 0;
+                load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
             }
         }
     }
