@@ -63,7 +63,7 @@ size_t gemm_workspace_floats_per_warp();
 
 // The persistent round: per-width preparation and the cooperative launch.
 // The node table travels as the kernel's parameter block (host buffer of
-// round_persistent_params_size() bytes, at most 300 nodes per launch).
+// round_persistent_params_size() bytes, at most 360 nodes per launch).
 int round_persistent_params_size();
 int round_persistent_max_nodes();
 size_t round_persistent_temp_floats(const GemmArgs* nodes, int n);
