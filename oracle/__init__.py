@@ -61,6 +61,8 @@ def _load():
                                  _P, _I64, _P, _P]
     lib.or_gateup_silu.argtypes = [_P, ctypes.c_int, _P, _P, ctypes.c_float, _P, _P,
                                    ctypes.c_float, _I64, _I64, _P, _P, _P, _P, _P]
+    lib.or_topk.argtypes = [_P, ctypes.c_int, _I64, _I64, ctypes.c_int, _P, _P]
+    lib.or_topk.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -162,3 +164,22 @@ def silu_tolerance(G, U, AG, AU, gscale_g=None, gscale_u=None):
     Bg = gemm_tolerance(AG)
     Bu = gemm_tolerance(AU)
     return 2.0 ** -8 * np.abs(h) + np.abs(dsilu) * np.abs(U) * Bg + np.abs(silu) * Bu + 1e-6
+
+
+def topk(logits: np.ndarray, k: int, V: int | None = None):
+    """Top-k of each row of an FP32 [M][ldv] array over its first V columns.
+
+    ignis README, "What sets it apart", "Speculative decoding (DFlash2)": the
+    top-k after the output head.  Returns (vals float32 [M][k], idx int32
+    [M][k]), best first: IEEE totalOrder with -0 == +0, equal values by lower
+    index.
+    """
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    M, ldv = logits.shape
+    V = ldv if V is None else int(V)
+    vals = np.empty((M, k), np.float32)
+    idx = np.empty((M, k), np.int32)
+    rc = _load().or_topk(_ptr(logits), M, V, ldv, int(k), _ptr(vals), _ptr(idx))
+    if rc != 0:
+        raise ValueError(f"oracle topk: bad arguments (M={M}, V={V}, ldv={ldv}, k={k})")
+    return vals, idx

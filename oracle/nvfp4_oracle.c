@@ -26,7 +26,8 @@
  * definition; all arithmetic is double; sums run in plain k order.
  * Parity status: every function here is pinned by tests (tables against
  * closed forms and torch's float8_e4m3fn; GEMM against closed forms and a
- * brute-force loop on tiny shapes).
+ * brute-force loop on tiny shapes; top-k against hand-derived cases, numpy's
+ * lexsort / stable argsort and its defining invariants).
  */
 #include <math.h>
 #include <stdint.h>
@@ -184,4 +185,83 @@ void or_gateup_silu(const uint16_t* X, int M,
         double g = G[i];
         H[i] = g / (1.0 + exp(-g)) * U[i];
     }
+}
+
+/* ------------------------------------------------------------------------
+ * Top-k over rows of FP32 logits (ignis README, "What sets it apart",
+ * "Speculative decoding (DFlash2)": the row-split top-k that follows the
+ * output head and gives a bit-identical answer).
+ *
+ * For each row m < M: the k largest of logits[m][0..V) (row stride ldv),
+ * written as vals[m][j], idx[m][j] for j = 0..k-1, best first.  "Largest"
+ * is IEEE 754 totalOrder except that -0 and +0 count as equal; equal
+ * values rank by lower index.  So for numbers (infinities included) it is
+ * the numeric order; a NaN with sign 0 ranks above +inf and one with sign 1
+ * below -inf; among NaNs of one sign a larger payload is further from the
+ * numbers.  The answer is unique.  Plain method: sort every index of the
+ * row with that comparison and keep the first k.
+ * ---------------------------------------------------------------------- */
+#include <stdlib.h>
+
+typedef struct {
+    float v;
+    int64_t i;
+} or_entry;
+
+/* -1 if x ranks before y (x is "larger"), +1 if after, 0 if tied. */
+static int or_value_rank(float x, float y)
+{
+    const int xn = isnan(x), yn = isnan(y);
+    if (!xn && !yn) {
+        if (x > y) return -1;
+        if (x < y) return 1;
+        return 0; /* equal numbers, -0 == +0 included */
+    }
+    uint32_t bx, by;
+    memcpy(&bx, &x, 4);
+    memcpy(&by, &y, 4);
+    /* class: 2 = NaN with sign 0, 1 = a number, 0 = NaN with sign 1 */
+    const int cx = xn ? ((bx >> 31) ? 0 : 2) : 1;
+    const int cy = yn ? ((by >> 31) ? 0 : 2) : 1;
+    if (cx != cy) return cx > cy ? -1 : 1;
+    /* two NaNs of the same sign: compare payloads (the 23 fraction bits) */
+    const uint32_t px = bx & 0x7FFFFFu, py = by & 0x7FFFFFu;
+    if (px == py) return 0;
+    if (cx == 2) return px > py ? -1 : 1; /* positive NaNs: larger payload ranks first */
+    return px > py ? 1 : -1;              /* negative NaNs: larger payload ranks last */
+}
+
+static int or_entry_cmp(const void* a, const void* b)
+{
+    const or_entry* x = (const or_entry*)a;
+    const or_entry* y = (const or_entry*)b;
+    const int r = or_value_rank(x->v, y->v);
+    if (r != 0) return r;
+    return (x->i < y->i) ? -1 : (x->i > y->i ? 1 : 0);
+}
+
+/* Returns 0, or -1 on bad arguments (k < 1, k > V, ldv < V) or no memory. */
+int or_topk(const float* logits, int M, int64_t V, int64_t ldv, int k, float* vals, int32_t* idx)
+{
+    if (M < 1 || V < 1 || k < 1 || k > V || ldv < V) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : bad)
+    for (int m = 0; m < M; ++m) {
+        or_entry* e = (or_entry*)malloc((size_t)V * sizeof(or_entry));
+        if (!e) {
+            bad |= 1;
+            continue;
+        }
+        for (int64_t i = 0; i < V; ++i) {
+            e[i].v = logits[(int64_t)m * ldv + i];
+            e[i].i = i;
+        }
+        qsort(e, (size_t)V, sizeof(or_entry), or_entry_cmp);
+        for (int j = 0; j < k; ++j) {
+            vals[(int64_t)m * k + j] = e[j].v;
+            idx[(int64_t)m * k + j] = (int32_t)e[j].i;
+        }
+        free(e);
+    }
+    return bad ? -1 : 0;
 }
