@@ -329,6 +329,47 @@ def round_io_bytes(r, M):
     return total
 
 
+def topk_detail(logits, dev, hbm_peak):
+    """Device time of nvfp4_topk on the round's own head logits (FP32
+    [8][151,936]), for rows 1 and 8 and k = 1, 8, 64: 50 calls captured in a
+    CUDA graph, replayed 5 times, timed with CUDA events.  The logits were
+    just written by the head, so they are L2-resident, as in a round."""
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi
+    out = []
+    V = logits.shape[1]
+    s = torch.cuda.Stream(device=dev)
+    for rows in (1, 8):
+        for k in (1, 8, 64):
+            x = logits[:rows]
+            vals = torch.empty((rows, k), dtype=torch.float32, device=dev)
+            idx = torch.empty((rows, k), dtype=torch.int32, device=dev)
+            with torch.cuda.stream(s):
+                abi.topk(x, k, values=vals, indices=idx, stream=s)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(50):
+                    abi.topk(x, k, values=vals, indices=idx, stream=s)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(s):
+                g.replay()
+                e0.record(s)
+                for _ in range(5):
+                    g.replay()
+                e1.record(s)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / 250
+            nbytes = rows * V * 4 + rows * k * 8
+            st, splits, slice_ = abi.nvfp4_topk_splits(rows, V, k, torch.cuda.get_device_properties(dev).multi_processor_count)
+            out.append({"rows": rows, "V": V, "k": k, "us": us, "GBps": nbytes / (us * 1e-6) / 1e9,
+                        "frac": nbytes / (us * 1e-6) / 1e9 / hbm_peak, "splits": splits, "slice": slice_})
+            del g
+    return {"kernel": "topk_kernel", "l2": "logits L2-resident (just written by the head, as in a round)",
+            "bytes": "rows*V*4 logits read + rows*k*8 written", "cases": out}
+
+
 def run_gemm_case(args):
     """Three direct nvfp4_gemm_decode / nvfp4_gemm_gateup_silu calls on one workload matrix."""
     import torch
@@ -451,6 +492,12 @@ def run_ours(args):
                 "kernel": ("round_kernel (persistent round, one launch per round)" if args.round_mode == "persistent"
                            else "decode_gemm_kernel (one launch per round node)")}
 
+    topk = None
+    if rank == 0 and not args.no_sweep:
+        rnd.replay(8, stream)
+        torch.cuda.synchronize()
+        topk = topk_detail(r.bufs["logits"], dev, hbm_peak)
+
     sweep = None
     if rank == 0 and not args.no_sweep:
         del rnd
@@ -484,6 +531,7 @@ def run_ours(args):
             "gpu_launches": graph_nodes * args.steps,
             "clocks": clk,
             "gemm_sweep": sweep,
+            "topk": topk,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

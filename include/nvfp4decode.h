@@ -210,6 +210,46 @@ NVFP4_API int nvfp4_round_replay_host(nvfp4_round* r, int M, const void* x_host,
 NVFP4_API int nvfp4_round_destroy(nvfp4_round* r);
 
 /*
+ * Top-k over rows of FP32 logits: the step after the output head (ignis
+ * README, "What sets it apart", "Speculative decoding (DFlash2)": the
+ * drafter's top-k over the vocabulary, replaced by a row-split kernel with
+ * a bit-identical answer).
+ *
+ * For each row m < rows, the k largest of logits[m*ldv + 0 .. m*ldv + V),
+ * best first, into values[m*k + j] and indices[m*k + j] (j < k).  Ranking:
+ * IEEE 754 totalOrder, except that -0 and +0 are equal, and equal values
+ * rank by lower index.  So numbers (and infinities) rank by value; a NaN
+ * with sign 0 ranks above +inf and one with sign 1 below -inf.  The answer
+ * is unique, and values are the input's own bits.
+ *
+ * Arguments: device pointers; logits 16-byte aligned with ldv % 4 == 0 and
+ * ldv >= V; values float[rows][k], indices int32[rows][k], 4-byte aligned.
+ * Limits: 1 <= rows <= NVFP4_TOPK_MAX_ROWS, 1 <= k <= NVFP4_TOPK_MAX_K,
+ * k <= V <= NVFP4_TOPK_MAX_V, and the row split must fit (S*k <= 16384,
+ * see nvfp4_topk_splits), else NVFP4_ERR_SHAPE.  Bad rows: NVFP4_ERR_M.
+ * Alignment: NVFP4_ERR_ALIGN.  NULL: NVFP4_ERR_ARG.
+ *
+ * One asynchronous launch on `stream`.  The library owns a per-device
+ * candidate workspace, allocated by the first call on a device (which must
+ * not be inside a stream capture: NVFP4_ERR_CAPTURE); later calls, captured
+ * or not, allocate nothing.  Calls on one device share that workspace and
+ * must be ordered (one stream, or synchronised).
+ */
+#define NVFP4_TOPK_MAX_ROWS 64
+#define NVFP4_TOPK_MAX_K 64
+#define NVFP4_TOPK_MAX_V (1 << 24)
+NVFP4_API int nvfp4_topk(const float* logits, int rows, int64_t V, int64_t ldv, int k, float* values,
+                         int32_t* indices, nvfp4_stream_t stream);
+
+/*
+ * Host helper (no GPU needed): the row split nvfp4_topk uses on a device
+ * with `sm_count` SMs -- `splits` slices per row of `slice` elements (a
+ * multiple of 4; the last slice may be shorter).  Returns the status the
+ * call itself would return for these sizes.
+ */
+NVFP4_API int nvfp4_topk_splits(int rows, int64_t V, int k, int sm_count, int* splits, int* slice);
+
+/*
  * Test aid: the dequantised weights exactly as the GEMM kernels form them,
  * W[n][k] = fp32(e2m1 * e4m3 * gscale), float [N][K] (unpadded).  Asynchronous.
  */

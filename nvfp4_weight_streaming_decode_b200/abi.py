@@ -33,6 +33,9 @@ NVFP4_ROUND_PERSISTENT = 0
 NVFP4_ROUND_CHAIN = 1
 NVFP4_DESC_GEMM = 0
 NVFP4_DESC_GATEUP_SILU = 1
+NVFP4_TOPK_MAX_ROWS = 64
+NVFP4_TOPK_MAX_K = 64
+NVFP4_TOPK_MAX_V = 1 << 24
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -58,6 +61,8 @@ _SIGNATURES = {
     "nvfp4_round_replay": (_I, [_P, _I, _P]),
     "nvfp4_round_replay_host": (_I, [_P, _I, _P, _P, _SZ, _P, _P, _SZ, _P]),
     "nvfp4_round_destroy": (_I, [_P]),
+    "nvfp4_topk": (_I, [_P, _I, _I64, _I64, _I, _P, _P, _P]),
+    "nvfp4_topk_splits": (_I, [_I, _I64, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "nvfp4_dequant_debug": (_I, [_P, _P, _F, _P, _I64, _I64, _P]),
     "nvfp4_unpack_debug": (_I, [_P, _P, _I64, _I64, _P, _P, _P]),
     "nvfp4_host_dequant_unit": (_I, [_P, _P, _F, _P]),
@@ -181,6 +186,17 @@ def nvfp4_round_destroy(handle):
     return load().nvfp4_round_destroy(handle)
 
 
+def nvfp4_topk(logits, rows, V, ldv, k, values, indices, stream):
+    return load().nvfp4_topk(logits, int(rows), int(V), int(ldv), int(k), values, indices, _s(stream))
+
+
+def nvfp4_topk_splits(rows, V, k, sm_count):
+    """(status, splits, slice) of the row split nvfp4_topk uses."""
+    sp, sl = _I(0), _I(0)
+    st = load().nvfp4_topk_splits(int(rows), int(V), int(k), int(sm_count), ctypes.byref(sp), ctypes.byref(sl))
+    return st, sp.value, sl.value
+
+
 def nvfp4_dequant_debug(wq_dev, ws_dev, gscale, W, N, K, stream):
     return load().nvfp4_dequant_debug(wq_dev, ws_dev, float(gscale), W, int(N), int(K), _s(stream))
 
@@ -258,6 +274,23 @@ def gemm_gateup_silu(X, wq_g, ws_g, gscale_g, wq_u, ws_u, gscale_u, Nff, K, H=No
                                  wq_u.data_ptr(), ws_u.data_ptr(), gscale_u, H.data_ptr(), Nff, K,
                                  _stream_ptr(stream)), "nvfp4_gemm_gateup_silu")
     return H
+
+
+def topk(logits, k, V=None, values=None, indices=None, stream=None):
+    """Top-k of each row of torch float32 [rows][ldv] device logits over the
+    first V columns: (values float32 [rows][k], indices int32 [rows][k])."""
+    import torch
+    rows, ldv = logits.shape
+    V = ldv if V is None else int(V)
+    if logits.stride(1) != 1:
+        raise ValueError("logits rows must be contiguous")
+    if values is None:
+        values = torch.empty((rows, k), dtype=torch.float32, device=logits.device)
+    if indices is None:
+        indices = torch.empty((rows, k), dtype=torch.int32, device=logits.device)
+    check(nvfp4_topk(logits.data_ptr(), rows, V, logits.stride(0), k, values.data_ptr(), indices.data_ptr(),
+                     _stream_ptr(stream)), "nvfp4_topk")
+    return values, indices
 
 
 def dequant_debug(wq, ws, gscale, N, K, stream=None):

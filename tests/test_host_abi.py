@@ -73,6 +73,39 @@ def test_argument_errors_return_before_any_cuda_call(lib):
     assert st == abi.NVFP4_ERR_ARG and not h
     badm = abi.Nvfp4GemmDesc(0, p, p, p, 1.0, None, None, 0.0, p, 32, 40)
     assert abi.nvfp4_round_create([badm])[0] == abi.NVFP4_ERR_SHAPE
+    # top-k over logits
+    assert abi.nvfp4_topk(None, 1, 100, 100, 1, p, p, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_topk(p, 0, 100, 100, 1, p, p, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_topk(p, 65, 100, 100, 1, p, p, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_topk(p, 1, 100, 100, 0, p, p, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_topk(p, 1, 100, 100, 65, p, p, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_topk(p, 1, 5, 8, 6, p, p, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_topk(p, 1, 100, 96, 1, p, p, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_topk(p, 1, (1 << 24) + 4, (1 << 24) + 4, 1, p, p, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_topk(p + 4, 1, 100, 100, 1, p, p, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_topk(p, 1, 100, 102, 1, p, p, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_topk(p, 1, 100, 100, 1, p + 2, p, None) == abi.NVFP4_ERR_ALIGN
+
+
+@pytest.mark.parametrize("rows", [1, 2, 3, 8, 13, 64])
+@pytest.mark.parametrize("V", [1, 3, 4, 5, 63, 255, 256, 257, 1000, 4099, 12289, 151936, 151937, 1 << 20, 3_000_000])
+@pytest.mark.parametrize("k", [1, 7, 8, 64])
+def test_topk_row_split(lib, rows, V, k):
+    """The row split of nvfp4_topk: slices a multiple of 4 long and at most
+    12,288 elements, none empty, covering the row; the merge (splits * k)
+    within 16,384 candidates; and an error exactly when no split fits."""
+    st, S, slice_ = abi.nvfp4_topk_splits(rows, V, k, 148)
+    if k > V:
+        assert st == abi.NVFP4_ERR_SHAPE
+        return
+    fits = any(sl <= 12288 and -(-V // sl) * k <= 16384 for sl in range(4, 12289, 4))
+    if not fits:
+        assert st == abi.NVFP4_ERR_SHAPE
+        return
+    assert st == abi.NVFP4_OK
+    assert slice_ % 4 == 0 and 4 <= slice_ <= 12288
+    assert (S - 1) * slice_ < V <= S * slice_
+    assert S * k <= 16384
 
 
 def _host_dequant(q, s, gscale):
