@@ -57,9 +57,9 @@ struct TopkParams {
 };
 
 struct SelectShared {
-    unsigned hist[256];
-    uint32_t sel_key[kSortSlots];
-    uint32_t sel_idx[kSortSlots];
+    unsigned hist[2][256];  // double-buffered: one pass fills one while the other is cleared
+    uint32_t sel_key[kSortSlots], sel_idx[kSortSlots];  // the winners, in arrival order
+    uint32_t out_key[kSortSlots], out_idx[kSortSlots];  // the winners, best first
     int digit, above, ties, count;
     int last;
 };
@@ -82,14 +82,10 @@ __device__ Select radix_select(int n, int want, Part part, SelectShared& sh)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t prefix = 0u, mask = 0u;
     Select r{0u, want, 0, false};
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        sh.hist[tid] = 0u;  // kTopkThreads == 256 bins
-        if (tid == 0) {
-            sh.digit = 0;
-            sh.above = 0;
-            sh.ties = 0;
-        }
-        __syncthreads();
+    sh.hist[0][tid] = 0u;  // kTopkThreads == 256 bins
+    __syncthreads();
+    int b = 0;
+    for (int shift = 24; shift >= 0; shift -= 8, b ^= 1) {
         for (int base = 0; base < n; base += kTopkThreads) {
             const int i = base + tid;
             uint32_t v = 0u;
@@ -97,7 +93,7 @@ __device__ Select radix_select(int n, int want, Part part, SelectShared& sh)
             if (i < n) ok = part(i, &v) && ((v & mask) == prefix);
             const unsigned d = ok ? ((v >> shift) & 255u) : 256u;
             const unsigned peers = __match_any_sync(0xffffffffu, d);
-            if (ok && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[d], (unsigned)__popc(peers));
+            if (ok && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[b][d], (unsigned)__popc(peers));
         }
         __syncthreads();
         if (warp == 0) {
@@ -105,7 +101,7 @@ __device__ Select radix_select(int n, int want, Part part, SelectShared& sh)
             unsigned c[8], local = 0u;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                c[j] = sh.hist[255 - 8 * lane - j];
+                c[j] = sh.hist[b][255 - 8 * lane - j];
                 local += c[j];
             }
             unsigned incl = local;
@@ -115,6 +111,12 @@ __device__ Select radix_select(int n, int want, Part part, SelectShared& sh)
                 if (lane >= off) incl += o;
             }
             const unsigned excl = incl - local;
+            if (lane == 0) {
+                sh.digit = 0;
+                sh.above = 0;
+                sh.ties = 0;
+            }
+            __syncwarp();
             if (excl < (unsigned)want && (unsigned)want <= incl) {
                 unsigned run = excl;
 #pragma unroll
@@ -127,10 +129,11 @@ __device__ Select radix_select(int n, int want, Part part, SelectShared& sh)
                     run += c[j];
                 }
             }
+        } else {
+            for (int j = tid - 32; j < 256; j += kTopkThreads - 32) sh.hist[b ^ 1][j] = 0u;  // for the next pass
         }
         __syncthreads();
         const int digit = sh.digit, above = sh.above, ties = sh.ties;
-        __syncthreads();  // everyone has read sh before it is written again
         prefix |= (uint32_t)digit << shift;
         mask |= 0xFFu << shift;
         want -= above;
@@ -142,11 +145,12 @@ __device__ Select radix_select(int n, int want, Part part, SelectShared& sh)
             break;
         }
     }
+    __syncthreads();  // every thread has read sh before anyone writes it again
     return r;
 }
 
 // Select the top `kk` (kk <= n, kk <= kSortSlots) of n elements given by
-// key(i) and idx(i), and leave them sorted, best first, in sh.sel_key/sel_idx.
+// key(i) and idx(i), and leave them best first in sh.out_key/out_idx.
 template <class KeyF, class IdxF>
 __device__ void block_topk(int n, int kk, KeyF key, IdxF idx, SelectShared& sh)
 {
@@ -169,8 +173,8 @@ __device__ void block_topk(int n, int kk, KeyF key, IdxF idx, SelectShared& sh)
     }
     if (tid == 0) sh.count = 0;
     if (tid < kSortSlots) {
-        sh.sel_key[tid] = 0u;
-        sh.sel_idx[tid] = kPadIdx;
+        sh.out_key[tid] = 0u;
+        sh.out_idx[tid] = kPadIdx;
     }
     __syncthreads();
     for (int i = tid; i < n; i += kTopkThreads) {
@@ -184,25 +188,18 @@ __device__ void block_topk(int n, int kk, KeyF key, IdxF idx, SelectShared& sh)
         }
     }
     __syncthreads();
-    // bitonic sort of the 64 slots, descending on (key, ~idx), by warp 0
-    if (tid < 32) {
-        for (int size = 2; size <= kSortSlots; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                const int lo = 2 * tid - (tid & (stride - 1));
-                const int hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const uint64_t a = ((uint64_t)sh.sel_key[lo] << 32) | (uint32_t)~sh.sel_idx[lo];
-                const uint64_t b = ((uint64_t)sh.sel_key[hi] << 32) | (uint32_t)~sh.sel_idx[hi];
-                if ((a < b) == desc) {
-                    const uint32_t tk = sh.sel_key[lo], ti = sh.sel_idx[lo];
-                    sh.sel_key[lo] = sh.sel_key[hi];
-                    sh.sel_idx[lo] = sh.sel_idx[hi];
-                    sh.sel_key[hi] = tk;
-                    sh.sel_idx[hi] = ti;
-                }
-                __syncwarp();
-            }
+    // Order the winners: each one's place is the number of winners that rank
+    // before it on (key, lower index); all of them are distinct.
+    const int cnt = sh.count < kSortSlots ? sh.count : kSortSlots;
+    if (tid < cnt) {
+        const uint32_t mk = sh.sel_key[tid], mi = sh.sel_idx[tid];
+        int rank = 0;
+        for (int j = 0; j < cnt; ++j) {
+            const uint32_t ok = sh.sel_key[j], oi = sh.sel_idx[j];
+            rank += (ok > mk || (ok == mk && oi < mi)) ? 1 : 0;
         }
+        sh.out_key[rank] = mk;
+        sh.out_idx[rank] = mi;
     }
     __syncthreads();
 }
@@ -243,8 +240,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p)
     uint32_t* ck = p.cand_key + (long long)m * kMergeCap + (long long)s * p.k;
     uint32_t* ci = p.cand_idx + (long long)m * kMergeCap + (long long)s * p.k;
     if (tid < p.k) {
-        ck[tid] = tid < kl ? sh.sel_key[tid] : 0u;
-        ci[tid] = tid < kl ? sh.sel_idx[tid] : kPadIdx - (uint32_t)(s * p.k + tid);
+        ck[tid] = tid < kl ? sh.out_key[tid] : 0u;
+        ci[tid] = tid < kl ? sh.out_idx[tid] : kPadIdx - (uint32_t)(s * p.k + tid);
     }
     // The CTA barrier orders every writer's stores before thread 0's release
     // (the count-in below); its acquire side orders the merge's loads after
@@ -272,7 +269,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p)
     block_topk(
         n2, p.k, [&](int i) { return mk[i]; }, [&](int i) { return mi[i]; }, sh);
     if (tid < p.k) {
-        const uint32_t id = sh.sel_idx[tid];
+        const uint32_t id = sh.out_idx[tid];
         // the input's own bits (-0 stays -0); an index past V cannot occur, but is never read
         p.indices[(long long)m * p.k + tid] = id < (uint32_t)p.V ? (int32_t)id : -1;
         p.values[(long long)m * p.k + tid] = id < (uint32_t)p.V ? row[id] : __int_as_float(0x7fffffff);
