@@ -20,8 +20,9 @@
  *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
  *    owns every buffer; the library never frees caller memory.
  *  - Device pointers must be 16-byte aligned (else NVFP4_ERR_ALIGN).
- *  - M in 1..8 (else NVFP4_ERR_M); N >= 1; K >= 16 and K % 16 == 0
- *    (else NVFP4_ERR_SHAPE).
+ *  - M in 1..8 (else NVFP4_ERR_M), except nvfp4_gemm_decode, which also
+ *    takes verify widths 9..64; N >= 1; K >= 16 and K % 16 == 0 (else
+ *    NVFP4_ERR_SHAPE).
  *  - X, Y and H are dense row-major with leading dimension K, N and N.
  *  - Calls never throw, abort or trap.  Asynchronous calls return once the
  *    work is enqueued on `stream`; a device fault surfaces at the caller's
@@ -51,7 +52,7 @@ typedef struct nvfp4_round nvfp4_round;     /* opaque graph-replay handle */
 enum {
     NVFP4_OK = 0,
     NVFP4_ERR_ARG = -1,       /* NULL pointer, bad kind, bad count */
-    NVFP4_ERR_M = -2,         /* M outside 1..8 */
+    NVFP4_ERR_M = -2,         /* M outside 1..8 (1..64 for nvfp4_gemm_decode) */
     NVFP4_ERR_SHAPE = -3,     /* N < 1, K < 16 or K % 16 != 0, size overflow */
     NVFP4_ERR_ALIGN = -4,     /* a device pointer is not 16-byte aligned */
     NVFP4_ERR_BAD_SCALE = -5, /* a scale byte is an E4M3 NaN code (0x7F / 0xFF) */
@@ -97,6 +98,13 @@ NVFP4_API int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon,
  * first call on a device allocates; that first call must not be made while
  * `stream` is being captured (NVFP4_ERR_CAPTURE).  Calls on one device that
  * overlap in time share that workspace and must not run concurrently.
+ *
+ * M: 1..8 decode lanes, or 9..64 rows at verify widths (README, "What sets
+ * it apart", "Speculative decoding (DFlash2)": lanes x (1 + drafts) rows
+ * verified in the same pass).  Widths 9..64 run on the tensor-memory kernel
+ * (its own per-device workspace, allocated by its first call under the same
+ * capture rule; nvfp4_verify_geometry describes its work split).  Other M:
+ * NVFP4_ERR_M.
  */
 NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                       float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);
@@ -116,8 +124,8 @@ NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, con
  * partial sums plus 10 KiB of counters, enough for 2,560 warps; every GPU
  * that loads the library holds it until the process exits.
  *
- * Arguments, layout and result are those of nvfp4_gemm_decode (the same
- * kernel runs).  The first call on a device resolves the array's device
+ * Arguments, layout and result are those of nvfp4_gemm_decode at M = 1..8
+ * (the same kernel runs); verify widths are not taken here (NVFP4_ERR_M).  The first call on a device resolves the array's device
  * address (cudaGetSymbolAddress) with that device current, so make that first
  * call before any stream capture.  Each call clears the arrival counters on
  * `stream` before the kernel.  All calls share the one array, which keeps the
@@ -275,6 +283,16 @@ NVFP4_API int nvfp4_host_dequant_unit(const uint8_t* q_unit, const uint8_t* s_un
 /* Host-side pack of one unit: canonical host planes -> one 1024 + 128 byte unit. */
 NVFP4_API int nvfp4_host_pack_unit(const uint8_t* wq_canon, const uint8_t* ws_canon, int64_t N, int64_t K,
                          int64_t tile, int64_t chunk, uint8_t* q_unit, uint8_t* s_unit);
+
+/*
+ * Host helper (no GPU needed): the work split nvfp4_gemm_decode uses at a
+ * verify width M (9..64) on a device with `sm_count` SMs -- `ctas` CTAs,
+ * each owning a contiguous range of the `units` (256-row tile pair, 64-column
+ * chunk) units -- and `nl`, the MMA's N (M padded to a multiple of 16).
+ * Returns NVFP4_ERR_M / NVFP4_ERR_SHAPE exactly when the call would.
+ */
+NVFP4_API int nvfp4_verify_geometry(int M, int64_t N, int64_t K, int sm_count, int64_t* ctas, int64_t* units,
+                                    int* nl);
 
 /* Text for a status code (static storage). */
 NVFP4_API const char* nvfp4_status_string(int status);

@@ -36,6 +36,7 @@ NVFP4_DESC_GATEUP_SILU = 1
 NVFP4_TOPK_MAX_ROWS = 64
 NVFP4_TOPK_MAX_K = 64
 NVFP4_TOPK_MAX_V = 1 << 24
+NVFP4_MAX_M = 64          # nvfp4_gemm_decode: 1..8 decode lanes, 9..64 verify rows
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -63,6 +64,8 @@ _SIGNATURES = {
     "nvfp4_round_destroy": (_I, [_P]),
     "nvfp4_topk": (_I, [_P, _I, _I64, _I64, _I, _P, _P, _P]),
     "nvfp4_topk_splits": (_I, [_I, _I64, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "nvfp4_verify_geometry": (_I, [_I, _I64, _I64, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                                   ctypes.POINTER(_I)]),
     "nvfp4_dequant_debug": (_I, [_P, _P, _F, _P, _I64, _I64, _P]),
     "nvfp4_unpack_debug": (_I, [_P, _P, _I64, _I64, _P, _P, _P]),
     "nvfp4_host_dequant_unit": (_I, [_P, _P, _F, _P]),
@@ -195,6 +198,14 @@ def nvfp4_topk_splits(rows, V, k, sm_count):
     sp, sl = _I(0), _I(0)
     st = load().nvfp4_topk_splits(int(rows), int(V), int(k), int(sm_count), ctypes.byref(sp), ctypes.byref(sl))
     return st, sp.value, sl.value
+
+
+def nvfp4_verify_geometry(M, N, K, sm_count):
+    """(status, ctas, units, nl) of the verify-width work split."""
+    c, u, nl = _I64(0), _I64(0), _I(0)
+    st = load().nvfp4_verify_geometry(int(M), int(N), int(K), int(sm_count), ctypes.byref(c), ctypes.byref(u),
+                                      ctypes.byref(nl))
+    return st, c.value, u.value, nl.value
 
 
 def nvfp4_dequant_debug(wq_dev, ws_dev, gscale, W, N, K, stream):

@@ -62,7 +62,10 @@ extern "C" int nvfp4_device_status(void)
     int v = 0;
     int st = nvfp4::read_and_clear_device_status(&v);
     if (st != NVFP4_OK) return st;
-    return v;
+    unsigned vv = 0;
+    st = nvfp4::read_and_clear_verify_status(&vv);
+    if (st != NVFP4_OK) return st;
+    return v | (int)(vv << 3);  // verify kernel: 8 = a streaming warp gave up, 16 = its MMA thread did
 }
 
 extern "C" int nvfp4_version(void) { return 100; }

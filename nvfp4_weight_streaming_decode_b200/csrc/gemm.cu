@@ -30,6 +30,7 @@
 
 #include <mutex>
 
+#include "async.cuh"
 #include "dequant.cuh"
 #include "internal.h"
 #include "layout.cuh"
@@ -41,7 +42,6 @@ __device__ unsigned int g_device_status;
 constexpr int kWarps = 16;                 // warps per CTA: one CTA per SM, so every warp has equal priority
 constexpr int kMinBlocks = 1;              // CTAs per SM the register budget is sized for
 constexpr int kSlotFloats = 512;           // partial-sum slot: 2 matrices x 32 rows x 8 lanes
-constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls before giving up
 
 struct KParams {
     const uint8_t* wq[2];
@@ -54,60 +54,6 @@ struct KParams {
     float* partials;
     unsigned* counters;
 };
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// All 32 lanes poll; gives up (returns false) after kWaitLimit rounds.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity)
-{
-    for (uint32_t it = 0; it < kWaitLimit; ++it)
-        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    return false;
-}
-
-__device__ __forceinline__ uint64_t evict_first_policy()
-{
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
-                                          uint64_t pol)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar), "l"(pol)
-        : "memory");
-}
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p)
 {
@@ -1215,6 +1161,8 @@ using namespace nvfp4;
 extern "C" int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                                  float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream)
 {
+    // verify widths run on the tensor-memory kernel
+    if (M >= kVerifyMinM && M <= kVerifyMaxM) return launch_verify(X, M, wq_dev, ws_dev, gscale, Y, N, K, (cudaStream_t)stream);
     GemmArgs a = {};
     a.kind = 0;
     a.X = X;

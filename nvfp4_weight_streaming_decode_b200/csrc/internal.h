@@ -75,4 +75,16 @@ int round_persistent_launch(void* params_host, unsigned* d_arrive, int M, int gr
 // Device-side status word (nonzero after a bounded wait gave up).
 int read_and_clear_device_status(int* status);
 
+// The decode GEMM at verify widths (M = kVerifyMinM..kVerifyMaxM) on the
+// tensor-memory path: geometry of a call, its launch, and its status word.
+constexpr int kVerifyMinM = 9, kVerifyMaxM = 64;
+struct VerifyGeometry {
+    long long n_tiles32, n_pairs, k_chunks, units, ctas;
+    int nl, tmem_cols;
+};
+int verify_geometry(int M, int64_t N, int64_t K, int sm_count, VerifyGeometry* g);
+int launch_verify(const void* X, int M, const uint8_t* wq, const uint8_t* ws, float gscale, float* Y, int64_t N,
+                  int64_t K, cudaStream_t stream);
+int read_and_clear_verify_status(unsigned* status);
+
 }  // namespace nvfp4

@@ -52,7 +52,11 @@ def test_packed_bytes(lib, N, K, ok):
 def test_argument_errors_return_before_any_cuda_call(lib):
     p = 1 << 20  # a fake, aligned "device" pointer: never dereferenced on these paths
     assert abi.nvfp4_gemm_decode(p, 0, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
-    assert abi.nvfp4_gemm_decode(p, 9, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_gemm_decode(p, 65, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_gemm_decode(p, 9, p, p, 1.0, p, 32, 40, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_gemm_decode(None, 20, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_gemm_decode(p + 8, 64, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_decode(p, 33, p, p, 1.0, p + 2, 32, 64, None) == abi.NVFP4_ERR_ALIGN
     assert abi.nvfp4_gemm_decode(p, 1, p, p, 1.0, p, 32, 40, None) == abi.NVFP4_ERR_SHAPE
     assert abi.nvfp4_gemm_decode(p, 1, p, p, 1.0, p, 0, 64, None) == abi.NVFP4_ERR_SHAPE
     assert abi.nvfp4_gemm_decode(None, 1, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ARG
@@ -159,3 +163,26 @@ def test_host_layout_model_every_code_with_every_scale(lib):
     W, _ = _host_dequant(q, s, 1.0)
     ref = oracle.dequant(q, s, 1.0)
     assert np.array_equal(W.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("M", [9, 16, 17, 33, 48, 64])
+@pytest.mark.parametrize("N,K", [(1, 16), (32, 64), (256, 512), (5120, 5120), (5120, 17408), (34816, 5120),
+                                 (151936, 5120), (1000, 1040)])
+def test_verify_geometry(lib, M, N, K):
+    """Work split of the verify-width kernel: every CTA owns a non-empty range
+    of (tile pair, chunk) units, at most two CTAs per SM, and the MMA's N is M
+    rounded up to 16."""
+    st, ctas, units, nl = abi.nvfp4_verify_geometry(M, N, K, 148)
+    assert st == abi.NVFP4_OK
+    pairs = -(-(-(-N // 32)) // 8)
+    assert units == pairs * -(-K // 64)
+    assert 1 <= ctas <= min(296, units)
+    assert nl % 16 == 0 and M <= nl < M + 16
+    assert all(units * (i + 1) // ctas > units * i // ctas for i in range(ctas))
+
+
+def test_verify_geometry_rejects():
+    assert abi.nvfp4_verify_geometry(8, 32, 64, 148)[0] == abi.NVFP4_ERR_M
+    assert abi.nvfp4_verify_geometry(65, 32, 64, 148)[0] == abi.NVFP4_ERR_M
+    assert abi.nvfp4_verify_geometry(16, 32, 40, 148)[0] == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_verify_geometry(16, 0, 64, 148)[0] == abi.NVFP4_ERR_SHAPE
