@@ -329,6 +329,55 @@ def round_io_bytes(r, M):
     return total
 
 
+def verify_sweep(dev, hbm_peak):
+    """The decode GEMM at verify widths (M = 9..64, the tensor-memory kernel),
+    timed on the device: for each workload and width, a CUDA graph of
+    back-to-back nvfp4_gemm_decode calls rotating through enough weight
+    copies to exceed L2, replayed under CUDA events."""
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi, synth
+    from nvfp4_weight_streaming_decode_b200.workloads import BYTES_PER_WEIGHT, make_matrix
+    out = []
+    s = torch.cuda.Stream(device=dev)
+    X = synth.torch_activations(1, 9, 64, 17408, dev)
+    cases = []
+    mats = [make_matrix(1, 700 + c, 5120, 5120, dev) for c in range(16)]
+    cases.append(("proj_n5120_k5120", [(m, 5120, 5120) for m in mats + mats]))
+    head = make_matrix(3, 0, 151936, 5120, dev, synth.EXP_LOGU_M6_4)
+    cases.append(("head_n151936_k5120", [(head, 151936, 5120)] * 4))
+    downs = [make_matrix(2, 800 + c, 5120, 17408, dev) for c in range(4)]
+    cases.append(("mlp_down_n5120_k17408", [(m, 5120, 17408) for m in downs + downs]))
+    for name, calls in cases:
+        N, K = calls[0][1], calls[0][2]
+        for M in (9, 16, 32, 64):
+            x = X[:M, :K].contiguous()
+            Y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            with torch.cuda.stream(s):
+                for (m, n_, k_) in calls:
+                    abi.gemm_decode(x, m.wq, m.ws, synth.GSCALE, n_, k_, Y=Y, stream=s)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for (m, n_, k_) in calls:
+                    abi.gemm_decode(x, m.wq, m.ws, synth.GSCALE, n_, k_, Y=Y, stream=s)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            with torch.cuda.stream(s):
+                g.replay()
+                e0.record(s)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(s)
+            e1.synchronize()
+            t = e0.elapsed_time(e1) * 1e-3 / reps / len(calls)
+            b = N * K * BYTES_PER_WEIGHT + 2 * M * K + 4 * M * N
+            out.append({"workload": name, "M": M, "us": t * 1e6, "GBps": b / t / 1e9, "frac": b / t / 1e9 / hbm_peak,
+                        "tflops": 2.0 * M * N * K / t / 1e12})
+            del g
+    return {"kernel": "verify_kernel (tcgen05.mma, accumulators in tensor memory)", "cases": out}
+
+
 def topk_detail(logits, dev, hbm_peak):
     """Device time of nvfp4_topk on the round's own head logits (FP32
     [8][151,936]), for rows 1 and 8 and k = 1, 8, 64: 50 calls captured in a
@@ -499,9 +548,11 @@ def run_ours(args):
         topk = topk_detail(r.bufs["logits"], dev, hbm_peak)
 
     sweep = None
+    verify = None
     if rank == 0 and not args.no_sweep:
         del rnd
         sweep = gemm_sweep(dev, hbm_peak)
+        verify = verify_sweep(dev, hbm_peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -532,6 +583,7 @@ def run_ours(args):
             "clocks": clk,
             "gemm_sweep": sweep,
             "topk": topk,
+            "verify_widths": verify,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

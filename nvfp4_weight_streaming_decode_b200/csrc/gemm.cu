@@ -780,7 +780,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) round_kernel(const RoundParams
         }
         if (!ok && lane == 0) atomicAnd(&cta_ok, 0);
         // Grid barrier: this CTA's warps meet, one thread counts the CTA in and
-        // waits for all CTAs, then releases the CTA.
+        // waits for all CTAs, then releases the CTA.  Every thread first makes
+        // its own output stores visible at GPU scope.
+        __threadfence();
         __syncthreads();
         if (threadIdx.x == 0) {
             __threadfence();

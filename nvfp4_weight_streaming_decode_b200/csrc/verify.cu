@@ -52,8 +52,9 @@ constexpr int kVTileRows = 128;                // MMA M
 constexpr int kVMaxNL = 64;                    // MMA N at most (M rows of X, padded to 16)
 constexpr int kABytes = kVTileRows * kChunkK * 2;  // one tile's bf16 A for one chunk: 16 KB
 constexpr int kXBytes = kVMaxNL * kChunkK * 2;     // one chunk of X: 8 KB
-constexpr int kVSlotFloats = kVMaxNL * 256;        // a partial: [64 m][256 rows] floats
+constexpr int kVSlotFloats = kVMaxNL * 256;        // a partial: [256 rows][64 m] floats
 constexpr int kVMaxPairs = 1 << 16;                // tile pairs a call may have (N <= 16.7M)
+constexpr int kVMaxSplit = 4;                      // CTAs per tile pair at most, on average
 
 // shared-memory map (bytes)
 constexpr int kOffA = 0;                                   // [2 buffers][2 tiles][16 KB]
@@ -230,6 +231,21 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
         // X and the outputs come from / go to the previous kernel's buffers
         asm volatile("griddepcontrol.wait;" ::: "memory");
 
+        // X pieces of this lane (16 bytes each; at most two per lane as nl <= 64)
+        auto load_x = [&](int jj, uint4 (&xr)[2]) {
+            const int cc = (int)((u0 + jj) % KC);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int pc = w * 32 + lane + h * kVWarps * 32;
+                xr[h] = make_uint4(0u, 0u, 0u, 0u);
+                const int nrow = pc >> 3, o = pc & 7;
+                const long long col = (long long)cc * kChunkK + 8 * o;
+                if (pc < p.NL * 8 && nrow < p.M && col < p.K)
+                    xr[h] = *reinterpret_cast<const uint4*>(p.X + nrow * p.K + col);
+            }
+        };
+        uint4 xnext[2];
+        load_x(0, xnext);
         const int g = lane >> 2, t = lane & 3;
         const int trow = 32 * (w & 3);  // first row of this warp in its 128-row tile
         const int tt = w >> 2;          // which tile of the pair
@@ -242,6 +258,9 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
             const long long t32 = pair * 8 + w;
             const bool valid = t32 < p.n_tiles32;
             const int slot = j % kVStages;
+            // this chunk's X was loaded one iteration ago; start the next chunk's now
+            const uint4 xcur[2] = {xnext[0], xnext[1]};
+            if (j + 1 < n) load_x(j + 1, xnext);
             uint32_t q[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
             uint32_t sw = 0u;
             if (valid) {
@@ -258,14 +277,11 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                 q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
                 q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
             }
-            // every lane has read the stage: refill it
-            __syncwarp();
-            if (lane == 0 && j + kVStages < n) issue(j + kVStages);
             const int b = j & 1;
             if (j >= 2 && !vwait(bars + 8 * (kBarEmpty + b), (uint32_t)(((j >> 1) - 1) & 1), abort)) {
                 if (lane == 0 && !*abort) vabort(abort, 1u);
                 pend_lo = j + 1;
-                pend_hi = (j + 1 + kVStages < n) ? j + 1 + kVStages : n;
+                pend_hi = (j + kVStages < n) ? j + kVStages : n;
                 break;
             }
             // A: this warp's 32 rows of its tile for this chunk, bf16, K-major core matrices
@@ -292,17 +308,22 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
             }
             // X: this chunk's 64 columns of every row (rows past M, columns past K: zero)
             const uint32_t xbuf = base + kOffX + b * kXBytes;
-            for (int pc = w * 32 + lane; pc < p.NL * 8; pc += kVWarps * 32) {
-                const int nrow = pc >> 3, o = pc & 7;
-                const long long col = (long long)c * kChunkK + 8 * o;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (nrow < p.M && col < p.K) v = *reinterpret_cast<const uint4*>(p.X + nrow * p.K + col);
-                st_shared_v4(xbuf + kmajor_off(nrow, o), v.x, v.y, v.z, v.w);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int pc = w * 32 + lane + h * kVWarps * 32;
+                if (pc < p.NL * 8)
+                    st_shared_v4(xbuf + kmajor_off(pc >> 3, pc & 7), xcur[h].x, xcur[h].y, xcur[h].z, xcur[h].w);
             }
-            // the tensor cores read A and X through the async proxy
+            // The tensor cores read A and X, and the next bulk copy writes this ring
+            // slot, through the async proxy: order this warp's shared-memory accesses
+            // first.  The slot is refilled only now, after the dequantisation above
+            // consumed every word read from it.
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if (lane == 0) mbar_arrive(bars + 8 * (kBarFull + b));
+            if (lane == 0) {
+                if (j + kVStages < n) issue(j + kVStages);
+                mbar_arrive(bars + 8 * (kBarFull + b));
+            }
 
             if (c == (int)KC - 1 || j == n - 1) {
                 // end of this pair's K range in this CTA: read the accumulators back
@@ -318,23 +339,26 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                 const long long row_g = t32 * 32 + lane;  // output row of this thread
                 const uint32_t taddr = tmem + ((uint32_t)(32 * (w & 3)) << 16) + (uint32_t)(tt * p.NL);
                 const int pslot = ps <= u0 ? 0 : 1;  // this CTA's first or last segment
-                float* pdst = p.part + (cta * 2 + pslot) * (long long)kVSlotFloats + (w * 32 + lane);
+                // a partial: this row's nl sums, contiguous ([256 rows][64] per slot)
+                float* pdst = p.part + (cta * 2 + pslot) * (long long)kVSlotFloats + (w * 32 + lane) * kVMaxNL;
                 for (int m0 = 0; m0 < p.NL; m0 += 16) {
                     uint32_t v[16];
                     tc_ld16(taddr + (uint32_t)m0, v);
+                    if (!whole) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int m = m0 + i;
-                        if (m < p.M) {
-                            const float a = __uint_as_float(v[i]);
-                            if (!whole)
-                                pdst[m * 256] = a;
-                            else if (row_g < p.N)
-                                p.Y[m * p.N + row_g] = (a * kEpilogueScale) * p.gscale;
-                        }
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<uint4*>(pdst + m0 + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    } else if (row_g < p.N) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (m0 + i < p.M) p.Y[(m0 + i) * p.N + row_g] = (__uint_as_float(v[i]) * kEpilogueScale) * p.gscale;
                     }
                 }
                 tc_fence_before();
+                // Partials go to another CTA: each lane makes its own stores visible at GPU
+                // scope before its warp signals (one thread's release does not cover the
+                // other warps' stores still in flight).
+                if (!whole) __threadfence();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars + 8 * kBarAccFree);
                 ++seg;
@@ -364,14 +388,32 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                     const int last = misc[2];
                     ++split;
                     if (last) {
+                        // every contributor's partial of this row, in CTA order, 16 sums at a time
                         const int glo_slot = vrange_begin(U, T, glo) >= ps ? 0 : 1;
-                        for (int m = 0; m < p.M; ++m) {
-                            float sum = 0.f;
+                        for (int m0 = 0; m0 < p.NL; m0 += 16) {
+                            float sum[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) sum[i] = 0.f;
                             for (long long ci = glo; ci <= ghi; ++ci) {
                                 const int sl = ci == glo ? glo_slot : 0;
-                                sum += __ldcg(p.part + (ci * 2 + sl) * (long long)kVSlotFloats + m * 256 + (w * 32 + lane));
+                                const float4* src = reinterpret_cast<const float4*>(
+                                    p.part + (ci * 2 + sl) * (long long)kVSlotFloats + (w * 32 + lane) * kVMaxNL + m0);
+                                float4 v4[4];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) v4[i] = __ldcg(src + i);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    sum[4 * i] += v4[i].x;
+                                    sum[4 * i + 1] += v4[i].y;
+                                    sum[4 * i + 2] += v4[i].z;
+                                    sum[4 * i + 3] += v4[i].w;
+                                }
                             }
-                            if (row_g < p.N) p.Y[m * p.N + row_g] = (sum * kEpilogueScale) * p.gscale;
+                            if (row_g < p.N) {
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    if (m0 + i < p.M) p.Y[(m0 + i) * p.N + row_g] = (sum[i] * kEpilogueScale) * p.gscale;
+                            }
                         }
                         if (w == 0 && lane == 0) p.counters[pair] = 0u;  // every contributor is in
                     }
@@ -499,7 +541,12 @@ int verify_geometry(int M, int64_t N, int64_t K, int sm_count, VerifyGeometry* g
     if (g->n_pairs > kVMaxPairs) return NVFP4_ERR_SHAPE;
     g->k_chunks = (K + kChunkK - 1) / kChunkK;
     g->units = g->n_pairs * g->k_chunks;
-    g->ctas = 2LL * sm_count < g->units ? 2LL * sm_count : g->units;
+    // two CTAs per SM, but no more than kVMaxSplit CTAs per tile pair on average: a pair
+    // split between more CTAs costs more in partial sums than the extra SMs stream
+    long long ctas = 2LL * sm_count;
+    if (ctas > g->n_pairs * kVMaxSplit) ctas = g->n_pairs * kVMaxSplit;
+    if (ctas > g->units) ctas = g->units;
+    g->ctas = ctas;
     g->nl = (M + 15) / 16 * 16;
     int cols = 32;
     while (cols < 2 * g->nl) cols *= 2;

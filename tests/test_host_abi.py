@@ -176,7 +176,7 @@ def test_verify_geometry(lib, M, N, K):
     assert st == abi.NVFP4_OK
     pairs = -(-(-(-N // 32)) // 8)
     assert units == pairs * -(-K // 64)
-    assert 1 <= ctas <= min(296, units)
+    assert 1 <= ctas <= min(296, units, 4 * pairs)
     assert nl % 16 == 0 and M <= nl < M + 16
     assert all(units * (i + 1) // ctas > units * i // ctas for i in range(ctas))
 
