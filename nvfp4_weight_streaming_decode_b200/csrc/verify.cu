@@ -213,11 +213,19 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
         const uint64_t pol = evict_first_policy();
         // stage j <-> unit x = u0 + j: this warp's 32-row tile of that unit's pair, one chunk
         auto tile_ok = [&](int j) { return ((u0 + j) / KC) * 8 + w < p.n_tiles32; };
-        auto issue = [&](int j) {  // lane 0
-            const long long x = u0 + j;
-            const long long t32 = (x / KC) * 8 + w;
+        // (pair, chunk) of unit u0 once; every later position advances incrementally
+        const long long pair0 = u0 / KC;
+        const int c0 = (int)(u0 - pair0 * KC);
+        long long ipair = pair0;  // the next stage to issue (lane 0), in stage order
+        int ic = c0;
+        auto issue = [&](int j) {  // lane 0; called for j = 0, 1, 2, ... in order
+            const long long t32 = ipair * 8 + w;
+            const long long unit = t32 * KC + ic;
+            if (++ic == (int)KC) {
+                ic = 0;
+                ++ipair;
+            }
             if (t32 >= p.n_tiles32) return;  // rows past N: no data, zeros below
-            const long long unit = t32 * KC + (x % KC);
             const int slot = j % kVStages;
             const uint32_t bar = rbar + 8 * slot;
             mbar_expect_tx(bar, (uint32_t)kUnitBytes);
@@ -232,8 +240,7 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
         asm volatile("griddepcontrol.wait;" ::: "memory");
 
         // X pieces of this lane (16 bytes each; at most two per lane as nl <= 64)
-        auto load_x = [&](int jj, uint4 (&xr)[2]) {
-            const int cc = (int)((u0 + jj) % KC);
+        auto load_x = [&](int cc, uint4 (&xr)[2]) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int pc = w * 32 + lane + h * kVWarps * 32;
@@ -244,23 +251,32 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                     xr[h] = *reinterpret_cast<const uint4*>(p.X + nrow * p.K + col);
             }
         };
-        uint4 xnext[2];
-        load_x(0, xnext);
+        auto store_x = [&](int bb, const uint4 (&xr)[2]) {
+            const uint32_t xb = base + kOffX + bb * kXBytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int pc = w * 32 + lane + h * kVWarps * 32;
+                if (pc < p.NL * 8) st_shared_v4(xb + kmajor_off(pc >> 3, pc & 7), xr[h].x, xr[h].y, xr[h].z, xr[h].w);
+            }
+        };
+        // X of the first chunk goes straight into buffer 0; every later chunk's X is
+        // loaded at the top of the iteration before it and stored at that iteration's
+        // end, once its buffer is free (the loads have landed by then).
+        uint4 xr[2];
+        load_x(c0, xr);
+        store_x(0, xr);
         const int g = lane >> 2, t = lane & 3;
         const int trow = 32 * (w & 3);  // first row of this warp in its 128-row tile
         const int tt = w >> 2;          // which tile of the pair
         int seg = 0, split = 0;
         int pend_lo = n, pend_hi = n;   // ring stages issued but not consumed, for the abort drain
+        long long pair = pair0;
+        int c = c0;
         for (int j = 0; j < n; ++j) {
-            const long long x = u0 + j;
-            const long long pair = x / KC;
-            const int c = (int)(x % KC);
             const long long t32 = pair * 8 + w;
             const bool valid = t32 < p.n_tiles32;
             const int slot = j % kVStages;
-            // this chunk's X was loaded one iteration ago; start the next chunk's now
-            const uint4 xcur[2] = {xnext[0], xnext[1]};
-            if (j + 1 < n) load_x(j + 1, xnext);
+            if (j + 1 < n) load_x(c + 1 == (int)KC ? 0 : c + 1, xr);  // stored into the next buffer at this iteration's end
             uint32_t q[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
             uint32_t sw = 0u;
             if (valid) {
@@ -277,13 +293,7 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                 q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
                 q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
             }
-            const int b = j & 1;
-            if (j >= 2 && !vwait(bars + 8 * (kBarEmpty + b), (uint32_t)(((j >> 1) - 1) & 1), abort)) {
-                if (lane == 0 && !*abort) vabort(abort, 1u);
-                pend_lo = j + 1;
-                pend_hi = (j + kVStages < n) ? j + kVStages : n;
-                break;
-            }
+            const int b = j & 1;  // buffer b is free: the previous iteration's end waited for it
             // A: this warp's 32 rows of its tile for this chunk, bf16, K-major core matrices
             const uint32_t abuf = base + kOffA + (b * 2 + tt) * kABytes;
             uint32_t S[2][2] = {{0u, 0u}, {0u, 0u}};
@@ -305,14 +315,6 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                 st_shared_v4(abuf + kmajor_off(row_lo, 2 * t + 1), a[2][0], a[2][2], a[3][0], a[3][2]);
                 st_shared_v4(abuf + kmajor_off(row_hi, 2 * t), a[0][1], a[0][3], a[1][1], a[1][3]);
                 st_shared_v4(abuf + kmajor_off(row_hi, 2 * t + 1), a[2][1], a[2][3], a[3][1], a[3][3]);
-            }
-            // X: this chunk's 64 columns of every row (rows past M, columns past K: zero)
-            const uint32_t xbuf = base + kOffX + b * kXBytes;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int pc = w * 32 + lane + h * kVWarps * 32;
-                if (pc < p.NL * 8)
-                    st_shared_v4(xbuf + kmajor_off(pc >> 3, pc & 7), xcur[h].x, xcur[h].y, xcur[h].z, xcur[h].w);
             }
             // The tensor cores read A and X, and the next bulk copy writes this ring
             // slot, through the async proxy: order this warp's shared-memory accesses
@@ -419,6 +421,22 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                     }
                 }
             }
+            // the next chunk's buffers: wait until the MMAs that last read them are done,
+            // then store its X (rows past M, columns past K: zero)
+            if (j + 1 < n) {
+                const int b1 = (j + 1) & 1;
+                if (j + 1 >= 2 && !vwait(bars + 8 * (kBarEmpty + b1), (uint32_t)((((j + 1) >> 1) - 1) & 1), abort)) {
+                    if (lane == 0 && !*abort) vabort(abort, 1u);
+                    pend_lo = j + 1;
+                    pend_hi = (j + 1 + kVStages < n) ? j + 1 + kVStages : n;
+                    break;
+                }
+                store_x(b1, xr);
+            }
+            if (++c == (int)KC) {
+                c = 0;
+                ++pair;
+            }
         }
         // after an abort: wait (bounded) for this warp's copies still in flight
         for (int s = pend_lo; s < pend_hi; ++s)
@@ -427,9 +445,9 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
         if (lane == 0) {
             int seg = 0;
             bool any = false;
+            int c = (int)(u0 % KC) - 1;
             for (int j = 0; j < n; ++j) {
-                const long long x = u0 + j;
-                const int c = (int)(x % KC);
+                if (++c == (int)KC) c = 0;
                 const int b = j & 1;
                 const bool first = j == 0 || c == 0;
                 if (!vwait1(bars + 8 * (kBarFull + b), (uint32_t)((j >> 1) & 1), abort)) {
