@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 METRIC = "NVFP4 decode GEMM HBM GB/s and % of B200 peak at M=1..8; full round ms"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["gemm.cu", "dequant.cuh", "layout.cuh"]
+KERNEL_SOURCES = ["gemm.cu", "dequant.cuh", "layout.cuh", "async.cuh"]
 
 
 def parse_args():
@@ -50,6 +50,8 @@ def parse_args():
                     help="only warm-up and timed replays (for an ncu launch list)")
     ap.add_argument("--gemm-case", default=None, choices=["head", "proj", "gateup", "down"],
                     help="only three direct calls of one workload GEMM at --width (for an ncu capture)")
+    ap.add_argument("--topk-case", type=int, default=None,
+                    help="only three top-k calls with this k over --width rows of 151,936 logits (for an ncu capture)")
     return ap.parse_args()
 
 
@@ -445,6 +447,23 @@ def run_gemm_case(args):
     return 0
 
 
+def run_topk_case(args):
+    """Three nvfp4_topk calls over [--width][151,936] seeded N(0,1) logits."""
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi, build
+    build.build()
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    x = torch.randn((args.width, 151936), generator=g, device=dev, dtype=torch.float32)
+    for _ in range(3):
+        abi.topk(x, args.topk_case)
+    torch.cuda.synchronize()
+    print(json.dumps({"topk_case": args.topk_case, "rows": args.width, "V": 151936, "ok": True}))
+    return 0
+
+
 def run_ours(args):
     import torch
 
@@ -598,6 +617,8 @@ def main():
         return run_reference(args)
     if args.gemm_case:
         return run_gemm_case(args)
+    if args.topk_case:
+        return run_topk_case(args)
     return run_ours(args)
 
 
