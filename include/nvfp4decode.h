@@ -285,6 +285,36 @@ NVFP4_API int nvfp4_host_pack_unit(const uint8_t* wq_canon, const uint8_t* ws_ca
                          int64_t tile, int64_t chunk, uint8_t* q_unit, uint8_t* s_unit);
 
 /*
+ * Grouped expert decode, one asynchronous launch (ignis, "Models and
+ * artifacts", the model table: Flash-Next has 512 routed experts per layer
+ * and ten chosen per token).  For every route (m, t), m < M lanes, t < T picks:
+ *   Y[(m*T + t)*N + n] = gscale_e * sum_k x[k] * w_e[n][k],  e = route[m*T + t],
+ *   x = X + m*K (x_per_route == 0: one input per lane, as for gate / up)
+ *     or X + (m*T + t)*K (x_per_route != 0: one input per route, as for down).
+ * experts[e] holds expert e's device-layout planes (nvfp4_pack_check) and
+ * global scale; every expert matrix is N x K.  An expert picked by several
+ * lanes is streamed once for all of them.  X bf16, Y float, route int32 and
+ * experts are device memory; route and experts may change between calls (and
+ * between graph replays).  Routes with a negative id give zero rows; ids >= E
+ * or experts whose planes are not 16-byte aligned also give zero rows and set
+ * bit 32 of nvfp4_device_status().  Results are deterministic.
+ * Limits: 1 <= M <= 8 (NVFP4_ERR_M), T >= 1 and M*T <= NVFP4_GROUPED_MAX_ROUTES
+ * (NVFP4_ERR_ARG), N <= 131,072 (NVFP4_ERR_SHAPE).  X 16-byte aligned, route
+ * and Y 4-byte, experts 8-byte (NVFP4_ERR_ALIGN).  Per-device workspace as for
+ * nvfp4_gemm_decode (first call outside any capture).
+ */
+typedef struct {
+    const uint8_t* wq; /* device-layout nibble plane */
+    const uint8_t* ws; /* device-layout scale plane */
+    float gscale;
+    int32_t reserved;
+} nvfp4_expert;
+#define NVFP4_GROUPED_MAX_ROUTES 128
+NVFP4_API int nvfp4_gemm_grouped(const void* X, int x_per_route, const int32_t* route, int M, int T,
+                                 const nvfp4_expert* experts, int E, float* Y, int64_t N, int64_t K,
+                                 nvfp4_stream_t stream);
+
+/*
  * Host helper (no GPU needed): the work split nvfp4_gemm_decode uses at a
  * verify width M (9..64) on a device with `sm_count` SMs -- `ctas` CTAs,
  * each owning a contiguous range of the `units` (256-row tile pair, 64-column

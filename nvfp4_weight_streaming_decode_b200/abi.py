@@ -36,6 +36,7 @@ NVFP4_DESC_GATEUP_SILU = 1
 NVFP4_TOPK_MAX_ROWS = 64
 NVFP4_TOPK_MAX_K = 64
 NVFP4_TOPK_MAX_V = 1 << 24
+NVFP4_GROUPED_MAX_ROUTES = 128
 NVFP4_MAX_M = 64          # nvfp4_gemm_decode: 1..8 decode lanes, 9..64 verify rows
 
 _P = ctypes.c_void_p
@@ -43,6 +44,10 @@ _I64 = ctypes.c_int64
 _SZ = ctypes.c_size_t
 _F = ctypes.c_float
 _I = ctypes.c_int
+
+
+class Nvfp4Expert(ctypes.Structure):
+    _fields_ = [("wq", _P), ("ws", _P), ("gscale", _F), ("reserved", ctypes.c_int32)]
 
 
 class Nvfp4GemmDesc(ctypes.Structure):
@@ -63,6 +68,7 @@ _SIGNATURES = {
     "nvfp4_round_replay_host": (_I, [_P, _I, _P, _P, _SZ, _P, _P, _SZ, _P]),
     "nvfp4_round_destroy": (_I, [_P]),
     "nvfp4_topk": (_I, [_P, _I, _I64, _I64, _I, _P, _P, _P]),
+    "nvfp4_gemm_grouped": (_I, [_P, _I, _P, _I, _I, _P, _I, _P, _I64, _I64, _P]),
     "nvfp4_topk_splits": (_I, [_I, _I64, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "nvfp4_verify_geometry": (_I, [_I, _I64, _I64, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                                    ctypes.POINTER(_I)]),
@@ -189,6 +195,11 @@ def nvfp4_round_destroy(handle):
     return load().nvfp4_round_destroy(handle)
 
 
+def nvfp4_gemm_grouped(X, x_per_route, route, M, T, experts, E, Y, N, K, stream):
+    return load().nvfp4_gemm_grouped(X, int(x_per_route), route, int(M), int(T), experts, int(E), Y, int(N), int(K),
+                                     _s(stream))
+
+
 def nvfp4_topk(logits, rows, V, ldv, k, values, indices, stream):
     return load().nvfp4_topk(logits, int(rows), int(V), int(ldv), int(k), values, indices, _s(stream))
 
@@ -285,6 +296,29 @@ def gemm_gateup_silu(X, wq_g, ws_g, gscale_g, wq_u, ws_u, gscale_u, Nff, K, H=No
                                  wq_u.data_ptr(), ws_u.data_ptr(), gscale_u, H.data_ptr(), Nff, K,
                                  _stream_ptr(stream)), "nvfp4_gemm_gateup_silu")
     return H
+
+
+def expert_table(mats, device):
+    """Device array of nvfp4_expert for a list of (wq, ws, gscale) device-layout planes."""
+    import numpy as np
+    import torch
+    rec = np.zeros((len(mats), 3), dtype=np.uint64)
+    for i, (wq, ws, gs) in enumerate(mats):
+        rec[i, 0] = wq.data_ptr()
+        rec[i, 1] = ws.data_ptr()
+        rec[i, 2] = int(np.float32(gs).view(np.uint32))  # gscale in the low 32 bits, reserved = 0
+    return torch.from_numpy(rec.view(np.int64)).to(device)
+
+
+def gemm_grouped(X, route, experts, E, N, K, x_per_route=False, Y=None, stream=None):
+    """Y float32 [M][T][N] for routes int32 [M][T] over the expert table (expert_table)."""
+    import torch
+    M, T = route.shape
+    if Y is None:
+        Y = torch.empty((M, T, N), dtype=torch.float32, device=X.device)
+    check(nvfp4_gemm_grouped(X.data_ptr(), 1 if x_per_route else 0, route.data_ptr(), M, T, experts.data_ptr(), E,
+                             Y.data_ptr(), N, K, _stream_ptr(stream)), "nvfp4_gemm_grouped")
+    return Y
 
 
 def topk(logits, k, V=None, values=None, indices=None, stream=None):

@@ -65,7 +65,12 @@ extern "C" int nvfp4_device_status(void)
     unsigned vv = 0;
     st = nvfp4::read_and_clear_verify_status(&vv);
     if (st != NVFP4_OK) return st;
-    return v | (int)(vv << 3);  // verify kernel: 8 = a streaming warp gave up, 16 = its MMA thread did
+    unsigned vg = 0;
+    st = nvfp4::read_and_clear_grouped_status(&vg);
+    if (st != NVFP4_OK) return st;
+    // verify kernel: 8 = a streaming warp gave up, 16 = its MMA thread did;
+    // grouped kernel: 32 = an invalid route, 64 = a bounded wait gave up
+    return v | (int)(vv << 3) | (int)(vg << 5);
 }
 
 extern "C" int nvfp4_version(void) { return 100; }

@@ -142,24 +142,6 @@ __device__ __forceinline__ void epilogue(const OutArgs& o, long long tile, const
 
 // One lane's share of a unit: X fragments are in xw; sq and ss point at the
 // lane's code bytes and scale word in shared memory.  Adds the unit's products into acc.
-__device__ __forceinline__ void mma_unit(const uint8_t* sq, const uint8_t* ss, const uint32_t (&xw)[8],
-                                         float (&acc)[2][4])
-{
-    const uint4 q0 = *reinterpret_cast<const uint4*>(sq);
-    const uint4 q1 = *reinterpret_cast<const uint4*>(sq + 512);
-    const uint32_t sw = *reinterpret_cast<const uint32_t*>(ss);
-    const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    uint32_t S[2][2];
-    scale_pairs(sw, S);
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            uint32_t a[4];
-            dequant_word(q[4 * r + s], S, r, a);
-            mma_bf16_16816(acc[r], a, xw[2 * s], xw[2 * s + 1]);
-        }
-}
 
 // Load one contributor's partial sums (this lane's NW*8 floats).
 template <int NW>

@@ -87,4 +87,7 @@ int launch_verify(const void* X, int M, const uint8_t* wq, const uint8_t* ws, fl
                   int64_t K, cudaStream_t stream);
 int read_and_clear_verify_status(unsigned* status);
 
+// Status word of the grouped expert kernel (1 = an invalid route, 2 = a bounded wait gave up).
+int read_and_clear_grouped_status(unsigned* status);
+
 }  // namespace nvfp4

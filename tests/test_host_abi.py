@@ -77,6 +77,16 @@ def test_argument_errors_return_before_any_cuda_call(lib):
     assert st == abi.NVFP4_ERR_ARG and not h
     badm = abi.Nvfp4GemmDesc(0, p, p, p, 1.0, None, None, 0.0, p, 32, 40)
     assert abi.nvfp4_round_create([badm])[0] == abi.NVFP4_ERR_SHAPE
+    # grouped expert decode
+    assert abi.nvfp4_gemm_grouped(None, 0, p, 2, 10, p, 512, p, 768, 2048, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_gemm_grouped(p, 0, p, 9, 10, p, 512, p, 768, 2048, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_gemm_grouped(p, 0, p, 8, 17, p, 512, p, 768, 2048, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_gemm_grouped(p, 0, p, 8, 10, p, 0, p, 768, 2048, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_gemm_grouped(p, 0, p, 8, 10, p, 512, p, 768, 2040, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_gemm_grouped(p, 0, p, 8, 10, p, 512, p, 131073, 2048, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_gemm_grouped(p + 8, 0, p, 8, 10, p, 512, p, 768, 2048, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_grouped(p, 0, p + 2, 8, 10, p, 512, p, 768, 2048, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_grouped(p, 0, p, 8, 10, p + 4, 512, p, 768, 2048, None) == abi.NVFP4_ERR_ALIGN
     # top-k over logits
     assert abi.nvfp4_topk(None, 1, 100, 100, 1, p, p, None) == abi.NVFP4_ERR_ARG
     assert abi.nvfp4_topk(p, 0, 100, 100, 1, p, p, None) == abi.NVFP4_ERR_M
