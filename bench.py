@@ -380,6 +380,59 @@ def verify_sweep(dev, hbm_peak):
     return {"kernel": "verify_kernel (tcgen05.mma, accumulators in tensor memory)", "cases": out}
 
 
+def grouped_sweep(dev, hbm_peak):
+    """Grouped expert decode (nvfp4_gemm_grouped) on 512 experts of the read
+    Flash-Next shape: gate/up-like 768 x 2,048 (one input per lane) and
+    down-like 2,048 x 768 (one input per route), for M = 1 and 8 lanes with 10
+    picks each.  A CUDA graph of 8 calls rotating through 8 seeded route tables
+    (so consecutive calls stream mostly different experts) is replayed under
+    CUDA events; GB/s counts the distinct selected experts' bytes per call."""
+    import numpy as np
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi, synth
+    from nvfp4_weight_streaming_decode_b200.workloads import BYTES_PER_WEIGHT, make_matrix
+    out = []
+    s = torch.cuda.Stream(device=dev)
+    E, T = 512, 10
+    for name, N, K, per_route in (("experts_768x2048", 768, 2048, False), ("experts_2048x768", 2048, 768, True)):
+        m = make_matrix(5, 0 if N == 768 else 1, E * N, K, dev)
+        kc = -(-K // 64)
+        qb, sb = (N // 32) * kc * 1024, (N // 32) * kc * 128
+        table = abi.expert_table([(m.wq[e * qb:(e + 1) * qb], m.ws[e * sb:(e + 1) * sb], synth.GSCALE)
+                                  for e in range(E)], dev)
+        for M in (1, 8):
+            rng = np.random.default_rng(M * 31 + N)
+            routes = [torch.from_numpy(np.stack([rng.choice(E, T, replace=False) for _ in range(M)]).astype(np.int32)).to(dev)
+                      for _ in range(8)]
+            uniq = np.mean([len(np.unique(r.cpu().numpy())) for r in routes])
+            X = synth.torch_activations(5, 2, M * T if per_route else M, K, dev)
+            Y = torch.empty((M, T, N), dtype=torch.float32, device=dev)
+            with torch.cuda.stream(s):
+                for r in routes:
+                    abi.gemm_grouped(X, r, table, E, N, K, x_per_route=per_route, Y=Y, stream=s)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for r in routes:
+                    abi.gemm_grouped(X, r, table, E, N, K, x_per_route=per_route, Y=Y, stream=s)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(s):
+                g.replay()
+                e0.record(s)
+                for _ in range(10):
+                    g.replay()
+                e1.record(s)
+            e1.synchronize()
+            t = e0.elapsed_time(e1) * 1e-3 / 80
+            b = uniq * N * K * BYTES_PER_WEIGHT
+            out.append({"workload": name, "M": M, "T": T, "experts_per_call": float(uniq), "us": t * 1e6,
+                        "GBps": b / t / 1e9, "frac": b / t / 1e9 / hbm_peak})
+            del g
+        del m, table
+    return {"kernel": "grouped_kernel", "cases": out}
+
+
 def topk_detail(logits, dev, hbm_peak):
     """Device time of nvfp4_topk on the round's own head logits (FP32
     [8][151,936]), for rows 1 and 8 and k = 1, 8, 64: 50 calls captured in a
@@ -568,10 +621,12 @@ def run_ours(args):
 
     sweep = None
     verify = None
+    grouped = None
     if rank == 0 and not args.no_sweep:
         del rnd
         sweep = gemm_sweep(dev, hbm_peak)
         verify = verify_sweep(dev, hbm_peak)
+        grouped = grouped_sweep(dev, hbm_peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -603,6 +658,7 @@ def run_ours(args):
             "gemm_sweep": sweep,
             "topk": topk,
             "verify_widths": verify,
+            "grouped_experts": grouped,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

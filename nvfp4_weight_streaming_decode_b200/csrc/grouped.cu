@@ -37,7 +37,9 @@ __device__ unsigned int g_grouped_status;
 namespace {
 
 constexpr int kGWarps = 16;     // one CTA of 16 warps per SM
-constexpr int kGStages = 6;     // per-warp ring, one unit per stage
+constexpr int kGStages = 3;     // per-warp ring depth
+constexpr int kGUPS = 4;        // units per stage (a stage crossing to the next expert takes one copy per part)
+constexpr int kGStage = kGUPS * kUnitBytes;
 constexpr int kGSlot = 256;     // a partial: 32 lanes x 8 floats
 constexpr int kGMaxTiles = 4096;  // 32-row tiles per expert (N <= 131,072)
 
@@ -67,6 +69,19 @@ __device__ __forceinline__ void g_ld_x32(const void* p, bool pred, uint32_t (&x)
 {
     asm volatile(
         "{\n .reg .pred q;\n setp.ne.u32 q, %9, 0;\n"
+        " mov.b32 %0, 0; mov.b32 %1, 0; mov.b32 %2, 0; mov.b32 %3, 0;\n"
+        " mov.b32 %4, 0; mov.b32 %5, 0; mov.b32 %6, 0; mov.b32 %7, 0;\n"
+        " @q ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%8];\n"
+        " @q ld.global.nc.v4.u32 {%4,%5,%6,%7}, [%8+16];\n}"
+        : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7])
+        : "l"(p), "r"((uint32_t)pred));
+}
+
+// The same without `volatile`, so the fast path's four loads can be issued
+// together (X is never written while the kernel runs).
+__device__ __forceinline__ void g_ld_x32_nv(const void* p, bool pred, uint32_t (&x)[8])
+{
+    asm("{\n .reg .pred q;\n setp.ne.u32 q, %9, 0;\n"
         " mov.b32 %0, 0; mov.b32 %1, 0; mov.b32 %2, 0; mov.b32 %3, 0;\n"
         " mov.b32 %4, 0; mov.b32 %5, 0; mov.b32 %6, 0; mov.b32 %7, 0;\n"
         " @q ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%8];\n"
@@ -142,9 +157,9 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
     __shared__ GroupTable gt;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long gw = (long long)blockIdx.x * kGWarps + warp;
-    const uint8_t* ring = gsm + warp * (kGStages * kUnitBytes);
-    const uint32_t ring_s = smem_addr(gsm) + warp * (kGStages * kUnitBytes);
-    const uint32_t bar_s = smem_addr(gsm + kGWarps * kGStages * kUnitBytes) + warp * kGStages * 8;
+    const uint8_t* ring = gsm + warp * (kGStages * kGStage);
+    const uint32_t ring_s = smem_addr(gsm) + warp * (kGStages * kGStage);
+    const uint32_t bar_s = smem_addr(gsm + kGWarps * kGStages * kGStage) + warp * kGStages * 8;
     if (lane == 0) {
         for (int s = 0; s < kGStages; ++s) mbar_init(bar_s + 8 * s);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -171,25 +186,36 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
     const long long KC = p.KC, UE = p.UE;
     const long long u0 = g_range_begin(U, TW, gw), u1 = g_range_begin(U, TW, gw + 1);
     const int n = (int)(u1 - u0);
+    const int n_stages = (n + kGUPS - 1) / kGUPS;
     const uint64_t pol = evict_first_policy();
 
     // issue cursor (lane 0): group and unit within the expert of the next stage
     int ig = (int)(u0 / UE);
     long long iul = u0 - ig * UE;
-    auto issue = [&](int j) {
-        const nvfp4_expert ex = p.experts[gt.g_expert[ig]];
+    auto issue = [&](int j) {  // stage j: units [u0 + 4j, ...), in stage order
         const int slot = j % kGStages;
         const uint32_t bar = bar_s + 8 * slot;
-        mbar_expect_tx(bar, (uint32_t)kUnitBytes);
-        bulk_load(ring_s + slot * kUnitBytes, ex.wq + iul * kUnitQ, kUnitQ, bar, pol);
-        bulk_load(ring_s + slot * kUnitBytes + kUnitQ, ex.ws + iul * kUnitS, kUnitS, bar, pol);
-        if (++iul == UE) {
-            iul = 0;
-            ++ig;
+        const int rem = n - j * kGUPS;
+        const int cnt = rem < kGUPS ? rem : kGUPS;
+        mbar_expect_tx(bar, (uint32_t)(cnt * kUnitBytes));
+        const uint32_t dst = ring_s + slot * kGStage;
+        for (int v = 0; v < cnt;) {
+            // the longest run of this stage's units within one expert
+            const long long left = UE - iul;
+            const int part = (long long)(cnt - v) < left ? cnt - v : (int)left;
+            const nvfp4_expert ex = p.experts[gt.g_expert[ig]];
+            bulk_load(dst + v * kUnitQ, ex.wq + iul * kUnitQ, part * kUnitQ, bar, pol);
+            bulk_load(dst + kGUPS * kUnitQ + v * kUnitS, ex.ws + iul * kUnitS, part * kUnitS, bar, pol);
+            v += part;
+            iul += part;
+            if (iul == UE) {
+                iul = 0;
+                ++ig;
+            }
         }
     };
     if (lane == 0) {
-        const int npre = n < kGStages ? n : kGStages;
+        const int npre = n_stages < kGStages ? n_stages : kGStages;
         for (int j = 0; j < npre; ++j) issue(j);
     }
 
@@ -219,88 +245,106 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[r][i] = 0.f;
     const long long first_tg = grp * (long long)p.tiles + tile;
-    for (int j = 0; j < n; ++j) {
-        const int slot = j % kGStages;
-        if (!warp_wait(bar_s + 8 * slot, (uint32_t)((j / kGStages) & 1))) {
+    int i = 0;  // units consumed
+    for (int js = 0; js < n_stages; ++js) {
+        const int slot = js % kGStages;
+        if (!warp_wait(bar_s + 8 * slot, (uint32_t)((js / kGStages) & 1))) {
             // give up: flag it, then wait (bounded) for the copies still in flight
             if (lane == 0) atomicOr(&g_grouped_status, 2u);
-            for (int j2 = j; j2 < n && j2 < j + kGStages; ++j2)
+            for (int j2 = js; j2 < n_stages && j2 < js + kGStages; ++j2)
                 warp_wait(bar_s + 8 * (j2 % kGStages), (uint32_t)((j2 / kGStages) & 1));
             return;
         }
-        const int col = chunk * kChunkK + 16 * t;
-        uint32_t xw[8];
-        g_ld_x32(xrow + col, xvalid && col < p.K, xw);
-        mma_unit(ring + slot * kUnitBytes + 16 * lane, ring + slot * kUnitBytes + kUnitQ + 4 * lane, xw, acc);
-        // the MMAs consumed every word read from the stage: refill it
-        __syncwarp();
-        if (lane == 0 && j + kGStages < n) issue(j + kGStages);
-
-        const bool tile_end = chunk == (int)KC - 1;
-        if (tile_end || j == n - 1) {
-            const long long tg = grp * (long long)p.tiles + tile;  // tile of the virtual matrix
-            const long long ts = tg * KC;
-            const long long glo = g_range_owner(U, TW, ts), ghi = g_range_owner(U, TW, ts + KC - 1);
-            bool write = true;
-            if (glo != ghi) {
-                const int slot_id = (tg == first_tg) ? 0 : 1;
-                float* dst = p.partials + ((size_t)gw * 2 + slot_id) * kGSlot + lane * 8;
-                reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-                reinterpret_cast<float4*>(dst)[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
-                __threadfence();
-                __syncwarp();
-                unsigned last = 0;
-                if (lane == 0) {
-                    unsigned old;
-                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + tg) : "memory");
-                    last = (old == (unsigned)(ghi - glo)) ? 1u : 0u;
+        const uint8_t* st = ring + slot * kGStage;
+        if (n - i > kGUPS && (int)KC - 1 - chunk >= kGUPS) {
+            // Fast path: four units inside one tile (so one group), none ending the
+            // tile or the range, and none in the last (possibly partial) chunk.
+            uint32_t xa[kGUPS][8];
+#pragma unroll
+            for (int v = 0; v < kGUPS; ++v) g_ld_x32_nv(xrow + (chunk + v) * kChunkK + 16 * t, xvalid, xa[v]);
+#pragma unroll
+            for (int v = 0; v < kGUPS; ++v)
+                mma_unit(st + v * kUnitQ + 16 * lane, st + kGUPS * kUnitQ + v * kUnitS + 4 * lane, xa[v], acc);
+            i += kGUPS;
+            chunk += kGUPS;
+        } else {
+#pragma unroll 1
+            for (int v = 0; v < kGUPS && i < n; ++v) {
+                const int col = chunk * kChunkK + 16 * t;
+                uint32_t xw[8];
+                g_ld_x32(xrow + col, xvalid && col < p.K, xw);
+                mma_unit(st + v * kUnitQ + 16 * lane, st + kGUPS * kUnitQ + v * kUnitS + 4 * lane, xw, acc);
+                ++i;
+                const bool tile_end = chunk == (int)KC - 1;
+                if (tile_end || i == n) {
+                const long long tg = grp * (long long)p.tiles + tile;  // tile of the virtual matrix
+                const long long ts = tg * KC;
+                const long long glo = g_range_owner(U, TW, ts), ghi = g_range_owner(U, TW, ts + KC - 1);
+                bool write = true;
+                if (glo != ghi) {
+                    const int slot_id = (tg == first_tg) ? 0 : 1;
+                    float* dst = p.partials + ((size_t)gw * 2 + slot_id) * kGSlot + lane * 8;
+                    reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+                    reinterpret_cast<float4*>(dst)[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+                    __threadfence();
+                    __syncwarp();
+                    unsigned last = 0;
+                    if (lane == 0) {
+                        unsigned old;
+                        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p.counters + tg) : "memory");
+                        last = (old == (unsigned)(ghi - glo)) ? 1u : 0u;
+                    }
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    write = last != 0;
+                    if (write) {
+                        // every contributor's partial, in warp order
+                        const int glo_slot = g_range_begin(U, TW, glo) >= ts ? 0 : 1;
+    #pragma unroll
+                        for (int r = 0; r < 2; ++r)
+    #pragma unroll
+                            for (int k = 0; k < 4; ++k) acc[r][k] = 0.f;
+                        for (long long w = glo; w <= ghi; ++w) {
+                            const int ws = (w == glo) ? glo_slot : 0;
+                            const float4* src = reinterpret_cast<const float4*>(p.partials + ((size_t)w * 2 + ws) * kGSlot + lane * 8);
+                            const float4 a = __ldcg(src), b = __ldcg(src + 1);
+                            acc[0][0] += a.x; acc[0][1] += a.y; acc[0][2] += a.z; acc[0][3] += a.w;
+                            acc[1][0] += b.x; acc[1][1] += b.y; acc[1][2] += b.z; acc[1][3] += b.w;
+                        }
+                        if (lane == 0) p.counters[tg] = 0u;  // every contributor is in
+                    }
                 }
-                last = __shfl_sync(0xffffffffu, last, 0);
-                write = last != 0;
                 if (write) {
-                    // every contributor's partial, in warp order
-                    const int glo_slot = g_range_begin(U, TW, glo) >= ts ? 0 : 1;
+    #pragma unroll
+                    for (int r = 0; r < 2; ++r)
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int m = 2 * t + (k & 1);
+                            const long long nrow = (long long)tile * kTileN + 16 * r + g8 + ((k & 2) ? 8 : 0);
+                            if (m < rows && nrow < p.N) {
+                                const int pos = gt.sorted[first + m];
+                                p.Y[pos * p.N + nrow] = (acc[r][k] * kEpilogueScale) * gscale;
+                            }
+                        }
+                }
 #pragma unroll
                     for (int r = 0; r < 2; ++r)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[r][i] = 0.f;
-                    for (long long w = glo; w <= ghi; ++w) {
-                        const int ws = (w == glo) ? glo_slot : 0;
-                        const float4* src = reinterpret_cast<const float4*>(p.partials + ((size_t)w * 2 + ws) * kGSlot + lane * 8);
-                        const float4 a = __ldcg(src), b = __ldcg(src + 1);
-                        acc[0][0] += a.x; acc[0][1] += a.y; acc[0][2] += a.z; acc[0][3] += a.w;
-                        acc[1][0] += b.x; acc[1][1] += b.y; acc[1][2] += b.z; acc[1][3] += b.w;
+                        for (int k = 0; k < 4; ++k) acc[r][k] = 0.f;
+                }
+                if (tile_end) {
+                    chunk = 0;
+                    if (++tile == p.tiles) {
+                        tile = 0;
+                        if (++grp < gt.n_groups) set_group();
                     }
-                    if (lane == 0) p.counters[tg] = 0u;  // every contributor is in
+                } else {
+                    ++chunk;
                 }
             }
-            if (write) {
-#pragma unroll
-                for (int r = 0; r < 2; ++r)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int m = 2 * t + (i & 1);
-                        const long long nrow = (long long)tile * kTileN + 16 * r + g8 + ((i & 2) ? 8 : 0);
-                        if (m < rows && nrow < p.N) {
-                            const int pos = gt.sorted[first + m];
-                            p.Y[pos * p.N + nrow] = (acc[r][i] * kEpilogueScale) * gscale;
-                        }
-                    }
-            }
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[r][i] = 0.f;
         }
-        if (tile_end) {
-            chunk = 0;
-            if (++tile == p.tiles) {
-                tile = 0;
-                if (++grp < gt.n_groups) set_group();
-            }
-        } else {
-            ++chunk;
-        }
+        // the MMAs above consumed every word read from the stage: refill it
+        __syncwarp();
+        if (lane == 0 && js + kGStages < n_stages) issue(js + kGStages);
     }
 }
 
@@ -337,7 +381,7 @@ int grouped_state(cudaStream_t stream, GroupedState** out)
     if (e == cudaSuccess) e = cudaMemset(counters, 0, n_counters * sizeof(unsigned));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kGWarps * kGStages * (kUnitBytes + 8));
+                                 kGWarps * kGStages * (kGStage + 8));
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         cudaFree(partials);
@@ -412,7 +456,7 @@ extern "C" int nvfp4_gemm_grouped(const void* X, int x_per_route, const int32_t*
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)gs->sm_count);
     cfg.blockDim = dim3(kGWarps * 32);
-    cfg.dynamicSmemBytes = (size_t)kGWarps * kGStages * (kUnitBytes + 8);
+    cfg.dynamicSmemBytes = (size_t)kGWarps * kGStages * (kGStage + 8);
     cfg.stream = (cudaStream_t)stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
