@@ -144,7 +144,9 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """One process per GPU (torchrun environment).  NCCL on GPUs; gloo when
+    asked for, or when no GPU is present (the CPU tests of this plumbing)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -153,8 +155,10 @@ def dist_setup(n_gpus):
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        be = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        if be == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(be, timeout=datetime.timedelta(seconds=300))
     return world, rank, local
 
 
@@ -165,13 +169,21 @@ def barrier(world):
 
 
 def max_over_ranks(value, world):
+    """The slowest rank's value (device time of the timed region)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_gbps(weight_bytes, steps, elapsed_s, world):
+    """Whole-job weight-stream rate: every replica streams weight_bytes per
+    step; the job takes the slowest rank's time."""
+    return world * weight_bytes * steps / elapsed_s / 1e9
 
 
 # ------------------------------------------------------------------ CPU oracle legs
@@ -579,7 +591,7 @@ def run_ours(args):
     clk = clocks.stop()
     elapsed_s = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world)
     ms_per_step = elapsed_s * 1e3 / args.steps
-    value = world * weight_bytes * args.steps / elapsed_s / 1e9
+    value = aggregate_gbps(weight_bytes, args.steps, elapsed_s, world)
 
     # end to end through the C ABI with host buffers: H2D of the layer-0 input,
     # the replay, D2H of the logits, every step
@@ -597,7 +609,7 @@ def run_ours(args):
         e1.record(stream)
     e1.synchronize()
     e2e_s = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world)
-    e2e_value = world * weight_bytes * e2e_steps / e2e_s / 1e9
+    e2e_value = aggregate_gbps(weight_bytes, e2e_steps, e2e_s, world)
 
     # roofline of the decode GEMM kernel over the round: every node is a launch of it
     launches = graph_nodes            # kernel launches per round: 1 (persistent) or one per GEMM node (chain)
