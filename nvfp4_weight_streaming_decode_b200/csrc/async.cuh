@@ -41,6 +41,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// The same test with a suspend-time hint: a thread whose phase is not yet
+// complete sleeps until it completes or `ns` nanoseconds pass, instead of
+// spinning (for waits that are often long).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // All 32 lanes poll; gives up (returns false) after kWaitLimit rounds.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity)
 {

@@ -10,21 +10,23 @@
 // At these widths the product no longer fits the register MMA path, so the
 // multiply runs on the fifth-generation tensor cores (tcgen05) with the
 // accumulators in tensor memory:
-//   * A CTA owns a contiguous range of (256-row tile pair, 64-column chunk)
-//     units -- stream-K at CTA granularity -- so every SM gets the same
-//     number of weight bytes, whatever the shape.
-//   * Eight dequantisation warps each stream one 32-row tile of the pair
+//   * A CTA (one per SM) owns a contiguous range of (512-row tile group,
+//     64-column chunk) units -- stream-K at CTA granularity -- so every SM
+//     gets the same number of weight bytes, whatever the shape.
+//   * Sixteen dequantisation warps each stream one 32-row tile of the group
 //     through their own ring of 1-D bulk copies, dequantise it exactly (the
 //     same bit placement and bf16 scale multiply as the M <= 8 kernel) and
 //     store it as bf16 into the MMA's K-major operand layout in shared
 //     memory; they also stage the chunk of X (the MMA's N side, M rows
 //     padded to a multiple of 16).  A and X are double-buffered.
-//   * One thread of a ninth warp issues tcgen05.mma (M = 128, N = 16..64,
-//     K = 16; four per tile and chunk) into two accumulators in tensor
-//     memory and commits each chunk to an mbarrier that frees its buffers.
-//   * At the end of a tile pair's K range the dequantisation warps read the
-//     accumulators back (tcgen05.ld) and write Y, or, for a pair split
-//     between CTAs, a partial sum; the last CTA to finish a split pair adds
+//   * One thread of a seventeenth warp issues tcgen05.mma (M = 128, N =
+//     16..64, K = 16; four per tile and chunk) into four accumulators in
+//     tensor memory and commits each chunk to an mbarrier that frees its
+//     buffers.  (The commit latency is paid once per chunk, so the more rows
+//     a chunk carries, the less of it shows.)
+//   * At the end of a tile group's K range the dequantisation warps read the
+//     accumulators back (tcgen05.ld) and write Y, or, for a group split
+//     between CTAs, a partial sum; the last CTA to finish a split group adds
 //     the partials in CTA order (deterministic) and writes Y.
 // Every wait is bounded; a wait that runs out flags the device status,
 // stops the CTA's work, waits (bounded) for its copies and MMAs in flight,
@@ -45,21 +47,24 @@ __device__ unsigned int g_verify_status;
 
 namespace {
 
-constexpr int kVWarps = 8;                     // dequantisation warps: 2 tiles x 4 x 32 rows
+constexpr int kVTiles = 4;                     // 128-row tiles per CTA group (512 rows)
+constexpr int kVWarps = 4 * kVTiles;           // dequantisation warps: one per 32-row tile
+constexpr int kVCtasPerSM = 1;                 // one CTA per SM: shared memory holds its operands
 constexpr int kVThreads = (kVWarps + 1) * 32;  // + the MMA / tensor-memory warp
 constexpr int kVStages = 3;                    // per-warp ring depth, one unit per stage
 constexpr int kVTileRows = 128;                // MMA M
 constexpr int kVMaxNL = 64;                    // MMA N at most (M rows of X, padded to 16)
 constexpr int kABytes = kVTileRows * kChunkK * 2;  // one tile's bf16 A for one chunk: 16 KB
 constexpr int kXBytes = kVMaxNL * kChunkK * 2;     // one chunk of X: 8 KB
-constexpr int kVSlotFloats = kVMaxNL * 256;        // a partial: [256 rows][64 m] floats
-constexpr int kVMaxPairs = 1 << 16;                // tile pairs a call may have (N <= 16.7M)
-constexpr int kVMaxSplit = 4;                      // CTAs per tile pair at most, on average
+constexpr int kVGroupRows = kVTiles * kVTileRows;  // 512
+constexpr int kVSlotFloats = kVMaxNL * kVGroupRows;  // a partial: [512 rows][64 m] floats
+constexpr int kVMaxPairs = 1 << 16;                // tile groups a call may have
+constexpr int kVMaxSplit = 4;                      // CTAs per tile group at most, on average
 
 // shared-memory map (bytes)
-constexpr int kOffA = 0;                                   // [2 buffers][2 tiles][16 KB]
-constexpr int kOffX = kOffA + 4 * kABytes;                 // [2 buffers][8 KB]
-constexpr int kOffRing = kOffX + 2 * kXBytes;              // [8 warps][3 stages][1152 B]
+constexpr int kOffA = 0;                                   // [2 buffers][kVTiles tiles][16 KB]
+constexpr int kOffX = kOffA + 2 * kVTiles * kABytes;       // [2 buffers][8 KB]
+constexpr int kOffRing = kOffX + 2 * kXBytes;              // [kVWarps warps][3 stages][1152 B]
 constexpr int kOffBar = kOffRing + kVWarps * kVStages * kUnitBytes;
 // barriers: ring[8][3], full[2], empty[2], acc, acc_free, part_done, last_ready, fin
 constexpr int kBarRing = 0, kBarFull = kVWarps * kVStages, kBarEmpty = kBarFull + 2, kBarAcc = kBarEmpty + 2,
@@ -144,11 +149,17 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Waits here are often long (operands, tensor-core commits), so the polls
+// sleep (up to kVSleepNs each) rather than spin and take issue slots from the
+// dequantisation warps; at most kVWaitLimit polls (about a second).
+constexpr uint32_t kVSleepNs = 1000;
+constexpr uint32_t kVWaitLimit = 1u << 20;
+
 // Bounded wait of a whole warp that also gives up once the CTA aborted.
 __device__ __forceinline__ bool vwait(uint32_t bar, uint32_t parity, const volatile int* abort)
 {
-    for (uint32_t it = 0; it < kWaitLimit; ++it) {
-        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    for (uint32_t it = 0; it < kVWaitLimit; ++it) {
+        if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, kVSleepNs))) return true;
         if (*abort) return false;
     }
     return false;
@@ -157,8 +168,8 @@ __device__ __forceinline__ bool vwait(uint32_t bar, uint32_t parity, const volat
 // The same for one thread.
 __device__ __forceinline__ bool vwait1(uint32_t bar, uint32_t parity, const volatile int* abort)
 {
-    for (uint32_t it = 0; it < kWaitLimit; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t it = 0; it < kVWaitLimit; ++it) {
+        if (mbar_try_wait_sleep(bar, parity, kVSleepNs)) return true;
         if (*abort) return false;
     }
     return false;
@@ -170,7 +181,7 @@ __device__ __forceinline__ void vabort(volatile int* abort, unsigned bit)
     atomicOr(&g_verify_status, bit);
 }
 
-__global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
+__global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VParams p)
 {
     extern __shared__ __align__(1024) uint8_t vsm[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -212,14 +223,14 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
         const uint32_t rbar = bars + 8 * (kBarRing + w * kVStages);
         const uint64_t pol = evict_first_policy();
         // stage j <-> unit x = u0 + j: this warp's 32-row tile of that unit's pair, one chunk
-        auto tile_ok = [&](int j) { return ((u0 + j) / KC) * 8 + w < p.n_tiles32; };
+        auto tile_ok = [&](int j) { return ((u0 + j) / KC) * kVWarps + w < p.n_tiles32; };
         // (pair, chunk) of unit u0 once; every later position advances incrementally
         const long long pair0 = u0 / KC;
         const int c0 = (int)(u0 - pair0 * KC);
         long long ipair = pair0;  // the next stage to issue (lane 0), in stage order
         int ic = c0;
         auto issue = [&](int j) {  // lane 0; called for j = 0, 1, 2, ... in order
-            const long long t32 = ipair * 8 + w;
+            const long long t32 = ipair * kVWarps + w;
             const long long unit = t32 * KC + ic;
             if (++ic == (int)KC) {
                 ic = 0;
@@ -273,7 +284,7 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
         long long pair = pair0;
         int c = c0;
         for (int j = 0; j < n; ++j) {
-            const long long t32 = pair * 8 + w;
+            const long long t32 = pair * kVWarps + w;
             const bool valid = t32 < p.n_tiles32;
             const int slot = j % kVStages;
             if (j + 1 < n) load_x(c + 1 == (int)KC ? 0 : c + 1, xr);  // stored into the next buffer at this iteration's end
@@ -295,7 +306,7 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
             }
             const int b = j & 1;  // buffer b is free: the previous iteration's end waited for it
             // A: this warp's 32 rows of its tile for this chunk, bf16, K-major core matrices
-            const uint32_t abuf = base + kOffA + (b * 2 + tt) * kABytes;
+            const uint32_t abuf = base + kOffA + (b * kVTiles + tt) * kABytes;
             uint32_t S[2][2] = {{0u, 0u}, {0u, 0u}};
             if (valid) scale_pairs(sw, S);
 #pragma unroll
@@ -341,7 +352,7 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                 const long long row_g = t32 * 32 + lane;  // output row of this thread
                 const uint32_t taddr = tmem + ((uint32_t)(32 * (w & 3)) << 16) + (uint32_t)(tt * p.NL);
                 const int pslot = ps <= u0 ? 0 : 1;  // this CTA's first or last segment
-                // a partial: this row's nl sums, contiguous ([256 rows][64] per slot)
+                // a partial: this row's nl sums, contiguous ([512 rows][64] per slot)
                 float* pdst = p.part + (cta * 2 + pslot) * (long long)kVSlotFloats + (w * 32 + lane) * kVMaxNL;
                 for (int m0 = 0; m0 < p.NL; m0 += 16) {
                     uint32_t v[16];
@@ -462,8 +473,8 @@ __global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const VParams p)
                 tc_fence_after();
                 const uint32_t xs = base + kOffX + b * kXBytes;
 #pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    const uint32_t as = base + kOffA + (b * 2 + tt) * kABytes;
+                for (int tt = 0; tt < kVTiles; ++tt) {
+                    const uint32_t as = base + kOffA + (b * kVTiles + tt) * kABytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc_mma(tmem + (uint32_t)(tt * p.NL), kmajor_desc(as + 256 * kk), kmajor_desc(xs + 256 * kk),
@@ -524,7 +535,7 @@ int verify_state(cudaStream_t stream, VerifyState** out)
     if (cs != cudaStreamCaptureStatusNone) return NVFP4_ERR_CAPTURE;
     int sms = 0;
     NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    const int max_ctas = 2 * sms;
+    const int max_ctas = kVCtasPerSM * sms;
     float* part = nullptr;
     unsigned* counters = nullptr;
     NVFP4_CUDA_TRY(cudaMalloc(&part, (size_t)max_ctas * 2 * kVSlotFloats * sizeof(float)));
@@ -555,19 +566,19 @@ int verify_geometry(int M, int64_t N, int64_t K, int sm_count, VerifyGeometry* g
     int st = check_shape(N, K);
     if (st != NVFP4_OK) return st;
     g->n_tiles32 = (N + kTileN - 1) / kTileN;
-    g->n_pairs = (g->n_tiles32 + 7) / 8;
+    g->n_pairs = (g->n_tiles32 + kVWarps - 1) / kVWarps;  // groups of kVWarps 32-row tiles
     if (g->n_pairs > kVMaxPairs) return NVFP4_ERR_SHAPE;
     g->k_chunks = (K + kChunkK - 1) / kChunkK;
     g->units = g->n_pairs * g->k_chunks;
-    // two CTAs per SM, but no more than kVMaxSplit CTAs per tile pair on average: a pair
+    // one CTA per SM, but no more than kVMaxSplit CTAs per tile group on average: a group
     // split between more CTAs costs more in partial sums than the extra SMs stream
-    long long ctas = 2LL * sm_count;
+    long long ctas = (long long)kVCtasPerSM * sm_count;
     if (ctas > g->n_pairs * kVMaxSplit) ctas = g->n_pairs * kVMaxSplit;
     if (ctas > g->units) ctas = g->units;
     g->ctas = ctas;
     g->nl = (M + 15) / 16 * 16;
     int cols = 32;
-    while (cols < 2 * g->nl) cols *= 2;
+    while (cols < kVTiles * g->nl) cols *= 2;
     g->tmem_cols = cols;
     return NVFP4_OK;
 }
