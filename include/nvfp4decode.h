@@ -317,7 +317,7 @@ NVFP4_API int nvfp4_gemm_grouped(const void* X, int x_per_route, const int32_t* 
 /*
  * Host helper (no GPU needed): the work split nvfp4_gemm_decode uses at a
  * verify width M (9..64) on a device with `sm_count` SMs -- `ctas` CTAs,
- * each owning a contiguous range of the `units` (256-row tile pair, 64-column
+ * each owning a contiguous range of the `units` (512-row tile group, 64-column
  * chunk) units -- and `nl`, the MMA's N (M padded to a multiple of 16).
  * Returns NVFP4_ERR_M / NVFP4_ERR_SHAPE exactly when the call would.
  */

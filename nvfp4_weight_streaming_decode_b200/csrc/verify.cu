@@ -50,6 +50,7 @@ namespace {
 constexpr int kVTiles = 4;                     // 128-row tiles per CTA group (512 rows)
 constexpr int kVWarps = 4 * kVTiles;           // dequantisation warps: one per 32-row tile
 constexpr int kVCtasPerSM = 1;                 // one CTA per SM: shared memory holds its operands
+constexpr int kVBufs = 2;                      // operand (A, X) buffers: chunks in flight to the tensor cores
 constexpr int kVThreads = (kVWarps + 1) * 32;  // + the MMA / tensor-memory warp
 constexpr int kVStages = 3;                    // per-warp ring depth, one unit per stage
 constexpr int kVTileRows = 128;                // MMA M
@@ -58,16 +59,16 @@ constexpr int kABytes = kVTileRows * kChunkK * 2;  // one tile's bf16 A for one 
 constexpr int kXBytes = kVMaxNL * kChunkK * 2;     // one chunk of X: 8 KB
 constexpr int kVGroupRows = kVTiles * kVTileRows;  // 512
 constexpr int kVSlotFloats = kVMaxNL * kVGroupRows;  // a partial: [512 rows][64 m] floats
-constexpr int kVMaxPairs = 1 << 16;                // tile groups a call may have
+constexpr int kVMaxGroups = 1 << 16;                // tile groups a call may have
 constexpr int kVMaxSplit = 4;                      // CTAs per tile group at most, on average
 
 // shared-memory map (bytes)
 constexpr int kOffA = 0;                                   // [2 buffers][kVTiles tiles][16 KB]
-constexpr int kOffX = kOffA + 2 * kVTiles * kABytes;       // [2 buffers][8 KB]
-constexpr int kOffRing = kOffX + 2 * kXBytes;              // [kVWarps warps][3 stages][1152 B]
+constexpr int kOffX = kOffA + kVBufs * kVTiles * kABytes;  // [kVBufs buffers][8 KB]
+constexpr int kOffRing = kOffX + kVBufs * kXBytes;         // [kVWarps warps][3 stages][1152 B]
 constexpr int kOffBar = kOffRing + kVWarps * kVStages * kUnitBytes;
 // barriers: ring[8][3], full[2], empty[2], acc, acc_free, part_done, last_ready, fin
-constexpr int kBarRing = 0, kBarFull = kVWarps * kVStages, kBarEmpty = kBarFull + 2, kBarAcc = kBarEmpty + 2,
+constexpr int kBarRing = 0, kBarFull = kVWarps * kVStages, kBarEmpty = kBarFull + kVBufs, kBarAcc = kBarEmpty + kVBufs,
               kBarAccFree = kBarAcc + 1, kBarPart = kBarAccFree + 1, kBarLast = kBarPart + 1,
               kBarFin = kBarLast + 1, kNumBars = kBarFin + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;            // tmem base, abort, last, pad
@@ -79,12 +80,12 @@ struct VParams {
     const uint16_t* X;
     float* Y;
     float* part;         // [ctas][2 slots][64][256]
-    unsigned* counters;  // [pairs]
+    unsigned* counters;  // [groups]
     float gscale;
     int M, NL, tmem_cols;
     long long N, K;
-    int KC, n_tiles32, n_pairs;
-    long long units, ctas;  // stream-K over units = n_pairs * KC
+    int KC, n_tiles32, n_groups;
+    long long units, ctas;  // stream-K over units = n_groups * KC
     uint32_t idesc;
 };
 
@@ -192,11 +193,11 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
     const long long U = p.units, T = p.ctas, KC = p.KC;
     const long long cta = blockIdx.x;
     const long long u0 = vrange_begin(U, T, cta), u1 = vrange_begin(U, T, cta + 1);
-    const int n = (int)(u1 - u0);  // this CTA's (pair, chunk) units; >= 1 as ctas <= units
+    const int n = (int)(u1 - u0);  // this CTA's (group, chunk) units; >= 1 as ctas <= units
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
-            const bool per_warp = (i == kBarFull || i == kBarFull + 1 || i == kBarAccFree || i == kBarPart);
+            const bool per_warp = (i >= kBarFull && i < kBarFull + kVBufs) || i == kBarAccFree || i == kBarPart;
             mbar_init(bars + 8 * i, per_warp ? (uint32_t)kVWarps : 1u);
         }
         misc[1] = 0;
@@ -222,19 +223,19 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
         const uint32_t ring_s = base + kOffRing + w * (kVStages * kUnitBytes);
         const uint32_t rbar = bars + 8 * (kBarRing + w * kVStages);
         const uint64_t pol = evict_first_policy();
-        // stage j <-> unit x = u0 + j: this warp's 32-row tile of that unit's pair, one chunk
+        // stage j <-> unit x = u0 + j: this warp's 32-row tile of that unit's group, one chunk
         auto tile_ok = [&](int j) { return ((u0 + j) / KC) * kVWarps + w < p.n_tiles32; };
-        // (pair, chunk) of unit u0 once; every later position advances incrementally
-        const long long pair0 = u0 / KC;
-        const int c0 = (int)(u0 - pair0 * KC);
-        long long ipair = pair0;  // the next stage to issue (lane 0), in stage order
+        // (group, chunk) of unit u0 once; every later position advances incrementally
+        const long long group0 = u0 / KC;
+        const int c0 = (int)(u0 - group0 * KC);
+        long long igroup = group0;  // the next stage to issue (lane 0), in stage order
         int ic = c0;
         auto issue = [&](int j) {  // lane 0; called for j = 0, 1, 2, ... in order
-            const long long t32 = ipair * kVWarps + w;
+            const long long t32 = igroup * kVWarps + w;
             const long long unit = t32 * KC + ic;
             if (++ic == (int)KC) {
                 ic = 0;
-                ++ipair;
+                ++igroup;
             }
             if (t32 >= p.n_tiles32) return;  // rows past N: no data, zeros below
             const int slot = j % kVStages;
@@ -278,13 +279,13 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
         store_x(0, xr);
         const int g = lane >> 2, t = lane & 3;
         const int trow = 32 * (w & 3);  // first row of this warp in its 128-row tile
-        const int tt = w >> 2;          // which tile of the pair
+        const int tt = w >> 2;          // which tile of the group
         int seg = 0, split = 0;
         int pend_lo = n, pend_hi = n;   // ring stages issued but not consumed, for the abort drain
-        long long pair = pair0;
+        long long group = group0;
         int c = c0;
         for (int j = 0; j < n; ++j) {
-            const long long t32 = pair * kVWarps + w;
+            const long long t32 = group * kVWarps + w;
             const bool valid = t32 < p.n_tiles32;
             const int slot = j % kVStages;
             if (j + 1 < n) load_x(c + 1 == (int)KC ? 0 : c + 1, xr);  // stored into the next buffer at this iteration's end
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                 q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
                 q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
             }
-            const int b = j & 1;  // buffer b is free: the previous iteration's end waited for it
+            const int b = j % kVBufs;  // buffer b is free: the previous iteration's end waited for it
             // A: this warp's 32 rows of its tile for this chunk, bf16, K-major core matrices
             const uint32_t abuf = base + kOffA + (b * kVTiles + tt) * kABytes;
             uint32_t S[2][2] = {{0u, 0u}, {0u, 0u}};
@@ -339,7 +340,7 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
             }
 
             if (c == (int)KC - 1 || j == n - 1) {
-                // end of this pair's K range in this CTA: read the accumulators back
+                // end of this group's K range in this CTA: read the accumulators back
                 if (!vwait(bars + 8 * kBarAcc, (uint32_t)(seg & 1), abort)) {
                     if (lane == 0 && !*abort) vabort(abort, 1u);
                     pend_lo = j + 1;
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                     break;
                 }
                 tc_fence_after();
-                const long long ps = pair * KC;  // the pair's first unit
+                const long long ps = group * KC;  // the group's first unit
                 const bool whole = ps >= u0 && ps + KC <= u1;
                 const long long row_g = t32 * 32 + lane;  // output row of this thread
                 const uint32_t taddr = tmem + ((uint32_t)(32 * (w & 3)) << 16) + (uint32_t)(tt * p.NL);
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                 if (lane == 0) mbar_arrive(bars + 8 * kBarAccFree);
                 ++seg;
                 if (!whole) {
-                    // count the CTA in on the pair; its last contributor adds every partial
+                    // count the CTA in on the group; its last contributor adds every partial
                     const long long glo = vrange_owner(U, T, ps), ghi = vrange_owner(U, T, ps + KC - 1);
                     if (lane == 0) mbar_arrive(bars + 8 * kBarPart);
                     if (w == 0) {
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                             unsigned old;
                             asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
                                          : "=r"(old)
-                                         : "l"(p.counters + pair)
+                                         : "l"(p.counters + group)
                                          : "memory");
                             misc[2] = (old == (unsigned)(ghi - glo)) ? 1 : 0;
                             mbar_arrive(bars + 8 * kBarLast);
@@ -428,15 +429,16 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                                     if (m0 + i < p.M) p.Y[(m0 + i) * p.N + row_g] = (sum[i] * kEpilogueScale) * p.gscale;
                             }
                         }
-                        if (w == 0 && lane == 0) p.counters[pair] = 0u;  // every contributor is in
+                        if (w == 0 && lane == 0) p.counters[group] = 0u;  // every contributor is in
                     }
                 }
             }
             // the next chunk's buffers: wait until the MMAs that last read them are done,
             // then store its X (rows past M, columns past K: zero)
             if (j + 1 < n) {
-                const int b1 = (j + 1) & 1;
-                if (j + 1 >= 2 && !vwait(bars + 8 * (kBarEmpty + b1), (uint32_t)((((j + 1) >> 1) - 1) & 1), abort)) {
+                const int b1 = (j + 1) % kVBufs;  // last used by chunk j + 1 - kVBufs
+                if (j + 1 >= kVBufs &&
+                    !vwait(bars + 8 * (kBarEmpty + b1), (uint32_t)((((j + 1) / kVBufs) - 1) & 1), abort)) {
                     if (lane == 0 && !*abort) vabort(abort, 1u);
                     pend_lo = j + 1;
                     pend_hi = (j + 1 + kVStages < n) ? j + 1 + kVStages : n;
@@ -446,7 +448,7 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
             }
             if (++c == (int)KC) {
                 c = 0;
-                ++pair;
+                ++group;
             }
         }
         // after an abort: wait (bounded) for this warp's copies still in flight
@@ -459,13 +461,13 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
             int c = (int)(u0 % KC) - 1;
             for (int j = 0; j < n; ++j) {
                 if (++c == (int)KC) c = 0;
-                const int b = j & 1;
+                const int b = j % kVBufs;
                 const bool first = j == 0 || c == 0;
-                if (!vwait1(bars + 8 * (kBarFull + b), (uint32_t)((j >> 1) & 1), abort)) {
+                if (!vwait1(bars + 8 * (kBarFull + b), (uint32_t)((j / kVBufs) & 1), abort)) {
                     if (!*abort) vabort(abort, 2u);
                     break;
                 }
-                // the previous pair's accumulators have been read back before they are overwritten
+                // the previous group's accumulators have been read back before they are overwritten
                 if (first && seg > 0 && !vwait1(bars + 8 * kBarAccFree, (uint32_t)((seg - 1) & 1), abort)) {
                     if (!*abort) vabort(abort, 2u);
                     break;
@@ -539,8 +541,8 @@ int verify_state(cudaStream_t stream, VerifyState** out)
     float* part = nullptr;
     unsigned* counters = nullptr;
     NVFP4_CUDA_TRY(cudaMalloc(&part, (size_t)max_ctas * 2 * kVSlotFloats * sizeof(float)));
-    cudaError_t e = cudaMalloc(&counters, (size_t)kVMaxPairs * sizeof(unsigned));
-    if (e == cudaSuccess) e = cudaMemset(counters, 0, (size_t)kVMaxPairs * sizeof(unsigned));
+    cudaError_t e = cudaMalloc(&counters, (size_t)kVMaxGroups * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemset(counters, 0, (size_t)kVMaxGroups * sizeof(unsigned));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kVSmemBytes);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -566,14 +568,14 @@ int verify_geometry(int M, int64_t N, int64_t K, int sm_count, VerifyGeometry* g
     int st = check_shape(N, K);
     if (st != NVFP4_OK) return st;
     g->n_tiles32 = (N + kTileN - 1) / kTileN;
-    g->n_pairs = (g->n_tiles32 + kVWarps - 1) / kVWarps;  // groups of kVWarps 32-row tiles
-    if (g->n_pairs > kVMaxPairs) return NVFP4_ERR_SHAPE;
+    g->n_groups = (g->n_tiles32 + kVWarps - 1) / kVWarps;  // groups of kVWarps 32-row tiles
+    if (g->n_groups > kVMaxGroups) return NVFP4_ERR_SHAPE;
     g->k_chunks = (K + kChunkK - 1) / kChunkK;
-    g->units = g->n_pairs * g->k_chunks;
+    g->units = g->n_groups * g->k_chunks;
     // one CTA per SM, but no more than kVMaxSplit CTAs per tile group on average: a group
     // split between more CTAs costs more in partial sums than the extra SMs stream
     long long ctas = (long long)kVCtasPerSM * sm_count;
-    if (ctas > g->n_pairs * kVMaxSplit) ctas = g->n_pairs * kVMaxSplit;
+    if (ctas > g->n_groups * kVMaxSplit) ctas = g->n_groups * kVMaxSplit;
     if (ctas > g->units) ctas = g->units;
     g->ctas = ctas;
     g->nl = (M + 15) / 16 * 16;
@@ -612,7 +614,7 @@ int launch_verify(const void* X, int M, const uint8_t* wq, const uint8_t* ws, fl
     p.K = K;
     p.KC = (int)geo.k_chunks;
     p.n_tiles32 = (int)geo.n_tiles32;
-    p.n_pairs = (int)geo.n_pairs;
+    p.n_groups = (int)geo.n_groups;
     p.units = geo.units;
     p.ctas = geo.ctas;
     // kind::f16 instruction: F32 accumulator, BF16 A and B, both K-major, N = nl, M = 128
@@ -643,7 +645,7 @@ int read_and_clear_verify_status(unsigned* status)
         NVFP4_CUDA_TRY(cudaGetDevice(&dev));
         std::lock_guard<std::mutex> lock(g_vmu);
         if (dev >= 0 && dev < 64 && g_vstate[dev].device == dev)
-            NVFP4_CUDA_TRY(cudaMemset(g_vstate[dev].counters, 0, (size_t)kVMaxPairs * sizeof(unsigned)));
+            NVFP4_CUDA_TRY(cudaMemset(g_vstate[dev].counters, 0, (size_t)kVMaxGroups * sizeof(unsigned)));
         NVFP4_CUDA_TRY(cudaDeviceSynchronize());
     }
     *status = v;
