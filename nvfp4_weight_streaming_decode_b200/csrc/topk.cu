@@ -60,6 +60,7 @@ struct SelectShared {
     unsigned hist[2][256];  // double-buffered: one pass fills one while the other is cleared
     uint32_t sel_key[kSortSlots], sel_idx[kSortSlots];  // the winners, in arrival order
     uint32_t out_key[kSortSlots], out_idx[kSortSlots];  // the winners, best first
+    uint64_t wc[8 * 16];                                // small-k path: each warp's best, as composites
     int digit, above, ties, count;
     int last;
 };
@@ -204,6 +205,85 @@ __device__ void block_topk(int n, int kk, KeyF key, IdxF idx, SelectShared& sh)
     __syncthreads();
 }
 
+// Small k (k <= KL <= 16): the same selection without histograms.  An
+// element's composite (key << 32 | ~index) orders it exactly as the ranking
+// does (larger is better) and is never 0, so 0 marks an empty slot.  Each
+// thread keeps its best KL composites sorted in registers; each warp then
+// takes its best kk in kk rounds of an arg-max across the lanes' list heads
+// (the winning lane shifts its list); warp 0 merges the eight warps' results
+// the same way.  Result: sh.out_key / out_idx, best first.
+template <int KL, class KeyF, class IdxF>
+__device__ void small_topk(int n, int kk, KeyF key, IdxF idx, SelectShared& sh)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint64_t L[KL];
+#pragma unroll
+    for (int j = 0; j < KL; ++j) L[j] = 0ull;
+    for (int i = tid; i < n; i += kTopkThreads) {
+        const uint64_t c = ((uint64_t)key(i) << 32) | (uint32_t)~idx(i);
+        if (c > L[KL - 1]) {
+#pragma unroll
+            for (int j = KL - 1; j > 0; --j) L[j] = c > L[j - 1] ? L[j - 1] : (c > L[j] ? c : L[j]);
+            L[0] = c > L[0] ? c : L[0];
+        }
+    }
+    if (tid < 8 * 16) sh.wc[tid] = 0ull;
+    __syncthreads();
+    uint64_t mine = 0ull;  // lane r keeps the warp's r-th best
+    for (int r = 0; r < kk; ++r) {
+        uint64_t best = L[0];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+            best = o > best ? o : best;
+        }
+        if (best != 0ull && L[0] == best) {
+#pragma unroll
+            for (int j = 0; j < KL - 1; ++j) L[j] = L[j + 1];
+            L[KL - 1] = 0ull;
+        }
+        if (lane == r) mine = best;
+    }
+    if (lane < kk) sh.wc[warp * KL + lane] = mine;
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int kPer = KL * (kTopkThreads / 32) / 32;  // candidates per lane
+        uint64_t C[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) C[q] = sh.wc[lane + 32 * q];
+        for (int r = 0; r < kk; ++r) {
+            uint64_t best = C[0];
+#pragma unroll
+            for (int q = 1; q < kPer; ++q) best = C[q] > best ? C[q] : best;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+                best = o > best ? o : best;
+            }
+#pragma unroll
+            for (int q = 0; q < kPer; ++q)
+                if (best != 0ull && C[q] == best) C[q] = 0ull;
+            if (lane == 0) {
+                sh.out_key[r] = (uint32_t)(best >> 32);
+                sh.out_idx[r] = ~(uint32_t)best;
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// The selection for kk winners, best first, in sh.out_key / out_idx.
+template <class KeyF, class IdxF>
+__device__ void select_topk(int n, int kk, KeyF key, IdxF idx, SelectShared& sh)
+{
+    if (kk <= 8)
+        small_topk<8>(n, kk, key, idx, sh);
+    else if (kk <= 16)
+        small_topk<16>(n, kk, key, idx, sh);
+    else
+        block_topk(n, kk, key, idx, sh);
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p)
 {
     extern __shared__ __align__(16) uint32_t tk_smem[];
@@ -233,7 +313,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p)
     }
     __syncthreads();
     const int kl = p.k < n ? p.k : n;
-    block_topk(
+    select_topk(
         n, kl, [&](int i) { return keys[i]; }, [&](int i) { return (uint32_t)(lo + i); }, sh);
 
     // 2. publish this slice's candidates (padding past kl ranks below every real element)
@@ -267,7 +347,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p)
         mi[i] = __ldcg(gi + i);
     }
     __syncthreads();
-    block_topk(
+    select_topk(
         n2, p.k, [&](int i) { return mk[i]; }, [&](int i) { return mi[i]; }, sh);
     if (tid < p.k) {
         const uint32_t id = sh.out_idx[tid];
