@@ -366,15 +366,16 @@ decode_gemm_kernel(const KParams p)
     int chunk = (int)(u0 - tile * KC);
     const int kc_last = (int)KC - 1;
     const int K32 = (int)p.K;
-    // X row of this lane (row 0 stands in past M; those lanes load nothing)
-    const uint16_t* xp = p.X + (long long)(g < M ? g : 0) * p.K + chunk * kChunkK + 16 * t;
+    // X row of this lane.  Past M a lane loads row g % M instead: it feeds only
+    // MMA output columns m >= M, which depend on nothing else and which the
+    // epilogue drops, and every lane then runs the same unpredicated loads.
+    const uint16_t* xp = p.X + (long long)(g % M) * p.K + chunk * kChunkK + 16 * t;
     int col = chunk * kChunkK + 16 * t;                 // this lane's first column in the unit
-    const bool x_lane = g < M;
     const uint32_t q_off = 16 * lane, s_off = 4 * lane;
     int slot = 0;
     uint32_t parity = 0;
     int i = 0;                                          // units consumed
-    uint32_t xf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // fast-path X (stays zero past M)
+    uint32_t xf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // fast-path X
     for (int j = 0; j < n_stages; ++j) {
         if (!warp_wait(bar_s + 8 * slot, parity)) {
             // Give up: flag it, then wait (bounded) for the copies still in flight.
@@ -397,7 +398,7 @@ decode_gemm_kernel(const KParams p)
             // needs a bounds, tile-end or range-end check.
 #pragma unroll
             for (int v = 0; v < UPS; ++v) {
-                ld_x32_keep(xp + v * kChunkK, x_lane, xf);
+                ld_x32_keep(xp + v * kChunkK, true, xf);
                 const uint8_t* sq = stage + v * kUnitQ + q_off;
                 const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
 #pragma unroll
@@ -411,9 +412,9 @@ decode_gemm_kernel(const KParams p)
 #pragma unroll 1
         for (int v = 0; v < UPS; ++v) {
             if (i < n_units) {
-                // This lane's 16 columns of X for lane row g (zeros past M or past K).
+                // This lane's 16 columns of X (zeros past K).
                 uint32_t xw[8];
-                ld_x32(xp, x_lane && col < K32, xw);
+                ld_x32(xp, col < K32, xw);
                 const uint8_t* sq = stage + v * kUnitQ + q_off;
                 const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
 #pragma unroll
