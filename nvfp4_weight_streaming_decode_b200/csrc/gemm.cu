@@ -182,8 +182,11 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         unsigned last = 0;
         if (lane == 0) {
             const unsigned others = (unsigned)(ghi - glo);
-            unsigned seen;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(o.counters + glo) : "memory");
+            // Leaving a tile in mid-range (no idle ring: gather_smem == 0), the
+            // warp is almost never the last contributor, so it counts in at once.
+            unsigned seen = ~0u;
+            if (gather_smem != 0)
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(o.counters + glo) : "memory");
             if (seen == others) {
                 last = 1u;
             } else {
@@ -612,9 +615,9 @@ __device__ __forceinline__ bool round_gemm(const RoundParams& rp, const RoundNod
     int chunk = (int)(u0 - tile * KC);
     const int kc_last = (int)KC - 1;
     const int K32 = nd.K;
-    const uint16_t* xp = static_cast<const uint16_t*>(nd.X) + (long long)(g < M ? g : 0) * nd.K + chunk * kChunkK + 16 * t;
+    // past M a lane loads row g % M, which feeds only dropped output columns
+    const uint16_t* xp = static_cast<const uint16_t*>(nd.X) + (long long)(g % M) * nd.K + chunk * kChunkK + 16 * t;
     int col = chunk * kChunkK + 16 * t;
-    const bool x_lane = g < M;
     const uint32_t q_off = 16 * lane, s_off = 4 * lane;
     uint32_t xf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     int i = 0;
@@ -625,7 +628,7 @@ __device__ __forceinline__ bool round_gemm(const RoundParams& rp, const RoundNod
         if (n_units - i > UPS && kc_last - chunk >= UPS) {
 #pragma unroll
             for (int v = 0; v < UPS; ++v) {
-                ld_x32_coherent(xp + v * kChunkK, x_lane, xf);
+                ld_x32_coherent(xp + v * kChunkK, true, xf);
                 mma_unit(stage + v * kUnitQ + q_off, stage + UPS * kUnitQ + v * kUnitS + s_off, xf, acc[0]);
             }
             i += UPS;
@@ -637,7 +640,7 @@ __device__ __forceinline__ bool round_gemm(const RoundParams& rp, const RoundNod
             for (int v = 0; v < UPS; ++v) {
                 if (i < n_units) {
                     uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                    ld_x32_coherent(xp, x_lane && col < K32, xw);
+                    ld_x32_coherent(xp, col < K32, xw);
                     mma_unit(stage + v * kUnitQ + q_off, stage + UPS * kUnitQ + v * kUnitS + s_off, xw, acc[0]);
                     ++i;
                     const bool tile_end = chunk == kc_last;

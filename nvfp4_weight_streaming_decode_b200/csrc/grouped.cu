@@ -228,13 +228,12 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
     int rows = 0, first = 0;
     float gscale = 0.f;
     const uint16_t* xrow = p.X;
-    bool xvalid = false;
     auto set_group = [&]() {
         rows = gt.g_rows[grp];
         first = gt.g_first[grp];
         gscale = p.experts[gt.g_expert[grp]].gscale;
-        xvalid = g8 < rows;
-        const int pos = gt.sorted[first + (xvalid ? g8 : 0)];
+        // past the group's rows a lane loads its first row, which feeds only dropped output columns
+        const int pos = gt.sorted[first + (g8 < rows ? g8 : 0)];
         xrow = p.X + (long long)(p.x_per_route ? pos : pos / p.T) * p.K;
     };
     set_group();
@@ -261,7 +260,7 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
             // tile or the range, and none in the last (possibly partial) chunk.
             uint32_t xa[kGUPS][8];
 #pragma unroll
-            for (int v = 0; v < kGUPS; ++v) g_ld_x32_nv(xrow + (chunk + v) * kChunkK + 16 * t, xvalid, xa[v]);
+            for (int v = 0; v < kGUPS; ++v) g_ld_x32_nv(xrow + (chunk + v) * kChunkK + 16 * t, true, xa[v]);
 #pragma unroll
             for (int v = 0; v < kGUPS; ++v)
                 mma_unit(st + v * kUnitQ + 16 * lane, st + kGUPS * kUnitQ + v * kUnitS + 4 * lane, xa[v], acc);
@@ -272,7 +271,7 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
             for (int v = 0; v < kGUPS && i < n; ++v) {
                 const int col = chunk * kChunkK + 16 * t;
                 uint32_t xw[8];
-                g_ld_x32(xrow + col, xvalid && col < p.K, xw);
+                g_ld_x32(xrow + col, col < p.K, xw);
                 mma_unit(st + v * kUnitQ + 16 * lane, st + kGUPS * kUnitQ + v * kUnitS + 4 * lane, xw, acc);
                 ++i;
                 const bool tile_end = chunk == (int)KC - 1;
