@@ -344,8 +344,9 @@ def round_io_bytes(r, M):
 
 
 def verify_sweep(dev, hbm_peak):
-    """The decode GEMM at verify widths (M = 9..64, the tensor-memory kernel),
-    timed on the device: for each workload and width, a CUDA graph of
+    """The decode GEMM at verify widths (M = 9..64: up to 32 on the decode
+    kernel with several lane blocks, above on the tensor-memory kernel), timed
+    on the device: for each workload and width, a CUDA graph of
     back-to-back nvfp4_gemm_decode calls rotating through enough weight
     copies to exceed L2, replayed under CUDA events."""
     import torch
@@ -364,7 +365,7 @@ def verify_sweep(dev, hbm_peak):
     cases.append(("mlp_down_n5120_k17408", [(m, 5120, 17408) for m in downs + downs]))
     for name, calls in cases:
         N, K = calls[0][1], calls[0][2]
-        for M in (9, 16, 32, 64):
+        for M in (9, 16, 24, 32, 40, 64):
             x = X[:M, :K].contiguous()
             Y = torch.empty((M, N), dtype=torch.float32, device=dev)
             with torch.cuda.stream(s):
@@ -387,9 +388,12 @@ def verify_sweep(dev, hbm_peak):
             t = e0.elapsed_time(e1) * 1e-3 / reps / len(calls)
             b = N * K * BYTES_PER_WEIGHT + 2 * M * K + 4 * M * N
             out.append({"workload": name, "M": M, "us": t * 1e6, "GBps": b / t / 1e9, "frac": b / t / 1e9 / hbm_peak,
-                        "tflops": 2.0 * M * N * K / t / 1e12})
+                        "tflops": 2.0 * M * N * K / t / 1e12,
+                        "kernel": ("decode_gemm_kernel, %d blocks of 8 lanes" % ((M + 7) // 8)) if M <= 32
+                        else "verify_kernel (tcgen05.mma, accumulators in tensor memory)"})
             del g
-    return {"kernel": "verify_kernel (tcgen05.mma, accumulators in tensor memory)", "cases": out}
+    return {"kernel": "M = 9..32: decode_gemm_kernel (bf16 m16n8k16, 2..4 lane blocks); "
+                      "M = 33..64: verify_kernel (tcgen05.mma, accumulators in tensor memory)", "cases": out}
 
 
 def grouped_sweep(dev, hbm_peak):

@@ -101,10 +101,11 @@ NVFP4_API int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon,
  *
  * M: 1..8 decode lanes, or 9..64 rows at verify widths (README, "What sets
  * it apart", "Speculative decoding (DFlash2)": lanes x (1 + drafts) rows
- * verified in the same pass).  Widths 9..64 run on the tensor-memory kernel
- * (its own per-device workspace, allocated by its first call under the same
- * capture rule; nvfp4_verify_geometry describes its work split).  Other M:
- * NVFP4_ERR_M.
+ * verified in the same pass).  Widths 9..32 run on the decode kernel with
+ * two to four blocks of 8 lanes sharing each dequantised word; widths 33..64
+ * run on the tensor-memory kernel (its own per-device workspace, allocated by
+ * its first call under the same capture rule; nvfp4_verify_geometry
+ * describes its work split).  Other M: NVFP4_ERR_M.
  */
 NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                       float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);

@@ -97,4 +97,32 @@ __device__ __forceinline__ void mma_unit(const uint8_t* sq, const uint8_t* ss, c
         }
 }
 
+// The same for NB blocks of 8 decode lanes (M up to 8 * NB): each word is
+// dequantised once and feeds one MMA per block; xw[b] and acc[b] belong to
+// lanes 8b..8b+7.
+template <int NB>
+__device__ __forceinline__ void mma_unit_nb(const uint8_t* sq, const uint8_t* ss, const uint32_t (&xw)[NB][8],
+                                            float (&acc)[NB][2][4])
+{
+    if constexpr (NB == 1) {
+        mma_unit(sq, ss, xw[0], acc[0]);
+    } else {
+        const uint4 q0 = *reinterpret_cast<const uint4*>(sq);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(sq + 512);
+        const uint32_t sw = *reinterpret_cast<const uint32_t*>(ss);
+        const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        uint32_t S[2][2];
+        scale_pairs(sw, S);
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                uint32_t a[4];
+                dequant_word(q[4 * r + s], S, r, a);
+#pragma unroll
+                for (int b = 0; b < NB; ++b) mma_bf16_16816(acc[b][r], a, xw[b][2 * s], xw[b][2 * s + 1]);
+            }
+    }
+}
+
 }  // namespace nvfp4

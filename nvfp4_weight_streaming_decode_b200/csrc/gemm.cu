@@ -43,6 +43,12 @@ constexpr int kWarps = 16;                 // warps per CTA: one CTA per SM, so 
 constexpr int kMinBlocks = 1;              // CTAs per SM the register budget is sized for
 constexpr int kSlotFloats = 512;           // partial-sum slot: 2 matrices x 32 rows x 8 lanes
 
+// Partial-sum slot stride for NA accumulator sets per lane (32 lanes x 8
+// floats each): kSlotFloats up to two sets, twice that up to four (kernels
+// with four sets run half as many warps, so the workspace holds them).
+template <int NA>
+constexpr int kSlotStride = NA <= 2 ? kSlotFloats : 2 * kSlotFloats;
+
 struct KParams {
     const uint8_t* wq[2];
     const uint8_t* ws[2];
@@ -117,19 +123,27 @@ struct OutArgs {
     float gs0, gs1;
 };
 
+// Accumulator sets per warp: one per matrix and block of 8 decode lanes.
 template <int M, int NW>
-__device__ __forceinline__ void epilogue(const OutArgs& o, long long tile, const float (&acc)[NW][2][4], int g,
-                                         int t)
+constexpr int kAccSets = NW * ((M + 7) / 8);
+
+template <int M, int NW>
+__device__ __forceinline__ void epilogue(const OutArgs& o, long long tile, const float (&acc)[kAccSets<M, NW>][2][4],
+                                         int g, int t)
 {
+    constexpr int NB = (M + 7) / 8;  // blocks of 8 decode lanes (plain GEMM only when more than one)
+    static_assert(NW == 1 || NB == 1, "the fused gate/up variant takes at most 8 lanes");
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int m = 2 * t + (i & 1);
+            const int m = 8 * b + 2 * t + (i & 1);
             const long long n = tile * kTileN + 16 * r + g + ((i & 2) ? 8 : 0);
             if (m < M && n < o.N) {
                 if (NW == 1) {
-                    static_cast<float*>(o.out)[m * o.N + n] = (acc[0][r][i] * kEpilogueScale) * o.gs0;
+                    static_cast<float*>(o.out)[m * o.N + n] = (acc[b][r][i] * kEpilogueScale) * o.gs0;
                 } else {
                     const float gv = (acc[0][r][i] * kEpilogueScale) * o.gs0;
                     const float uv = (acc[NW - 1][r][i] * kEpilogueScale) * o.gs1;
@@ -169,6 +183,7 @@ template <int M, int NW>
 __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane, uint32_t gather_smem,
                                        uint32_t gather_bytes, uint32_t gather_bar)
 {
+    constexpr int NA = kAccSets<M, NW>;  // accumulator sets per lane in a partial
     const long long U = o.units, TW = o.total_warps, KC = o.k_chunks;
     const long long ts = tile * KC, te = ts + KC;
     const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
@@ -199,15 +214,15 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         if (!last) return;
     }
     const int glo_slot = (range_begin(U, TW, glo) >= ts) ? 0 : 1;
-    float sum[NW][2][4];
+    float sum[NA][2][4];
 #pragma unroll
-    for (int a = 0; a < NW; ++a)
+    for (int a = 0; a < NA; ++a)
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int i = 0; i < 4; ++i) sum[a][r][i] = 0.f;
     const int C = (int)(ghi - glo + 1);
-    constexpr uint32_t kPartBytes = NW * 1024;  // the used part of a slot: 32 lanes x NW x 8 floats
+    constexpr uint32_t kPartBytes = NA * 1024;  // the used part of a slot: 32 lanes x NA x 8 floats
     // contributors 0..nb-1 through the ring, nb..C-1 through registers
     int nb = gather_smem != 0 ? (int)(gather_bytes / kPartBytes) : 0;
     if (nb > C) nb = C;
@@ -221,19 +236,19 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
             const long long w = glo + c;
             const int ws = (w == glo) ? glo_slot : 0;
             const uint64_t pol = evict_first_policy();
-            bulk_load(gather_smem + c * kPartBytes, o.partials + ((size_t)w * 2 + ws) * kSlotFloats, kPartBytes,
+            bulk_load(gather_smem + c * kPartBytes, o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA>, kPartBytes,
                       gather_bar, pol);
         }
     }
-    constexpr int kBatch = NW == 1 ? 4 : 2;  // contributors whose loads are in flight together (more costs the callers spills)
-    float4 v[kBatch][NW * 2];
+    constexpr int kBatch = NA == 1 ? 4 : NA == 2 ? 2 : 1;  // contributors whose loads are in flight together (more costs the callers spills)
+    float4 v[kBatch][NA * 2];
     long long w0 = glo + nb;
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
         const long long w = w0 + b;
         if (w <= ghi) {
             const int ws = (w == glo) ? glo_slot : 0;
-            load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
+            load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), v[b]);
         }
     }
     if (nb > 0) {
@@ -245,21 +260,21 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
             warp_wait(gather_bar, 0u);
         }
         for (int c = 0; c < nb; ++c) {
-            float4 x[NW * 2];
+            float4 x[NA * 2];
             if (gathered) {
-                const uint32_t src = gather_smem + c * kPartBytes + lane * (NW * 32);
+                const uint32_t src = gather_smem + c * kPartBytes + lane * (NA * 32);
 #pragma unroll
-                for (int k = 0; k < NW * 2; ++k)
+                for (int k = 0; k < NA * 2; ++k)
                     asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
                                  : "=f"(x[k].x), "=f"(x[k].y), "=f"(x[k].z), "=f"(x[k].w)
                                  : "r"(src + 16 * k));
             } else {
                 const long long w = glo + c;
                 const int ws = (w == glo) ? glo_slot : 0;
-                load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), x);
+                load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), x);
             }
 #pragma unroll
-            for (int k = 0; k < NW * 2; ++k) {
+            for (int k = 0; k < NA * 2; ++k) {
                 sum[k >> 1][k & 1][0] += x[k].x;
                 sum[k >> 1][k & 1][1] += x[k].y;
                 sum[k >> 1][k & 1][2] += x[k].z;
@@ -272,7 +287,7 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         for (int b = 0; b < kBatch; ++b) {
             if (w0 + b <= ghi) {
 #pragma unroll
-                for (int k = 0; k < NW * 2; ++k) {
+                for (int k = 0; k < NA * 2; ++k) {
                     sum[k >> 1][k & 1][0] += v[b][k].x;
                     sum[k >> 1][k & 1][1] += v[b][k].y;
                     sum[k >> 1][k & 1][2] += v[b][k].z;
@@ -287,7 +302,7 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
             const long long w = w0 + b;
             if (w <= ghi) {
                 const int ws = (w == glo) ? glo_slot : 0;
-                load_partial<NW>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * (NW * 8), v[b]);
+                load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), v[b]);
             }
         }
     }
@@ -297,18 +312,22 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
 
 // STAGES shared-memory stages per warp, each holding UPS consecutive units of
 // each of the NW matrices (one bulk copy per plane and matrix per stage).
-template <int M, int NW, int STAGES, int UPS>
-__global__ void __launch_bounds__(kWarps * 32, kMinBlocks)
+// W warps per CTA (one CTA per SM).  M up to 16: lanes 8..15 form a second
+// block of the MMA's 8-wide side, sharing every dequantised word.
+template <int M, int NW, int STAGES, int UPS, int W>
+__global__ void __launch_bounds__(W * 32, kMinBlocks)
 decode_gemm_kernel(const KParams p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int kMatStage = UPS * kUnitBytes;
     constexpr int kStage = NW * kMatStage;
+    constexpr int NB = (M + 7) / 8;        // blocks of 8 decode lanes
+    constexpr int NA = kAccSets<M, NW>;    // accumulator sets
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const long long gw = (long long)blockIdx.x * kWarps + warp;
+    const long long gw = (long long)blockIdx.x * W + warp;
 
     // Dependents may begin launching; they wait for this grid before using its results.
     asm volatile("griddepcontrol.launch_dependents;");
@@ -321,9 +340,9 @@ decode_gemm_kernel(const KParams p)
 
     uint8_t* ring = smem + warp * (STAGES * kStage);
     const uint32_t ring_s = smem_addr(ring);
-    const uint32_t bar_s = smem_addr(smem + kWarps * STAGES * kStage) + warp * STAGES * 8;
+    const uint32_t bar_s = smem_addr(smem + W * STAGES * kStage) + warp * STAGES * 8;
     // one more mbarrier per warp, for gathering partial sums into the idle ring
-    const uint32_t gather_bar = smem_addr(smem + kWarps * STAGES * (kStage + 8)) + warp * 8;
+    const uint32_t gather_bar = smem_addr(smem + W * STAGES * (kStage + 8)) + warp * 8;
 
     if (lane == 0) {
 #pragma unroll
@@ -356,9 +375,9 @@ decode_gemm_kernel(const KParams p)
     // Everything below reads X or writes outputs / workspace: wait for the producer grid.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    float acc[NW][2][4];
+    float acc[NA][2][4];
 #pragma unroll
-    for (int a = 0; a < NW; ++a)
+    for (int a = 0; a < NA; ++a)
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -373,12 +392,18 @@ decode_gemm_kernel(const KParams p)
     // MMA output columns m >= M, which depend on nothing else and which the
     // epilogue drops, and every lane then runs the same unpredicated loads.
     const uint16_t* xp = p.X + (long long)(g % M) * p.K + chunk * kChunkK + 16 * t;
+    // the second block's row, (8 + g) % M, as an offset from the first's
+    const long long x_delta = NB > 1 ? (long long)((8 + g) % M - g % M) * p.K : 0;
     int col = chunk * kChunkK + 16 * t;                 // this lane's first column in the unit
     const uint32_t q_off = 16 * lane, s_off = 4 * lane;
     int slot = 0;
     uint32_t parity = 0;
     int i = 0;                                          // units consumed
-    uint32_t xf[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // fast-path X
+    uint32_t xf[NB][8];                                 // fast-path X
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xf[b][k] = 0u;
     for (int j = 0; j < n_stages; ++j) {
         if (!warp_wait(bar_s + 8 * slot, parity)) {
             // Give up: flag it, then wait (bounded) for the copies still in flight.
@@ -401,11 +426,14 @@ decode_gemm_kernel(const KParams p)
             // needs a bounds, tile-end or range-end check.
 #pragma unroll
             for (int v = 0; v < UPS; ++v) {
-                ld_x32_keep(xp + v * kChunkK, true, xf);
+#pragma unroll
+                for (int b = 0; b < NB; ++b) ld_x32_keep(xp + b * x_delta + v * kChunkK, true, xf[b]);
                 const uint8_t* sq = stage + v * kUnitQ + q_off;
                 const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
 #pragma unroll
-                for (int mat = 0; mat < NW; ++mat) mma_unit(sq + mat * kMatStage, ss + mat * kMatStage, xf, acc[mat]);
+                for (int mat = 0; mat < NW; ++mat)
+                    mma_unit_nb<NB>(sq + mat * kMatStage, ss + mat * kMatStage, xf,
+                                    *reinterpret_cast<float(*)[NB][2][4]>(acc + mat * NB));
             }
             i += UPS;
             chunk += UPS;
@@ -416,20 +444,23 @@ decode_gemm_kernel(const KParams p)
         for (int v = 0; v < UPS; ++v) {
             if (i < n_units) {
                 // This lane's 16 columns of X (zeros past K).
-                uint32_t xw[8];
-                ld_x32(xp, col < K32, xw);
+                uint32_t xw[NB][8];
+#pragma unroll
+                for (int b = 0; b < NB; ++b) ld_x32(xp + b * x_delta, col < K32, xw[b]);
                 const uint8_t* sq = stage + v * kUnitQ + q_off;
                 const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
 #pragma unroll
-                for (int mat = 0; mat < NW; ++mat) mma_unit(sq + mat * kMatStage, ss + mat * kMatStage, xw, acc[mat]);
+                for (int mat = 0; mat < NW; ++mat)
+                    mma_unit_nb<NB>(sq + mat * kMatStage, ss + mat * kMatStage, xw,
+                                    *reinterpret_cast<float(*)[NB][2][4]>(acc + mat * NB));
                 ++i;
                 const bool tile_end = chunk == kc_last;
                 if (tile_end || i == n_units) {
                     // Partial slot: 0 for the tile this warp's range starts in, 1 for a later one.
                     const int slot_id = (tile == first_tile) ? 0 : 1;
-                    float* dst = p.partials + ((size_t)gw * 2 + slot_id) * kSlotFloats + lane * (NW * 8);
+                    float* dst = p.partials + ((size_t)gw * 2 + slot_id) * kSlotStride<NA> + lane * (NA * 8);
 #pragma unroll
-                    for (int a = 0; a < NW; ++a)
+                    for (int a = 0; a < NA; ++a)
 #pragma unroll
                         for (int r = 0; r < 2; ++r)
                             reinterpret_cast<float4*>(dst)[a * 2 + r] =
@@ -448,7 +479,7 @@ decode_gemm_kernel(const KParams p)
                     // in flight, so the ring can take the partial sums of a combine.
                     tile_done<M, NW>(o, tile, lane, i == n_units ? ring_s : 0u, STAGES * kStage, gather_bar);
 #pragma unroll
-                    for (int a = 0; a < NW; ++a)
+                    for (int a = 0; a < NA; ++a)
 #pragma unroll
                         for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -811,17 +842,29 @@ namespace {
 constexpr int kStagesPlain = 2, kUnitsPerStagePlain = 6;
 constexpr int kStagesFused = 2, kUnitsPerStageFused = 3;
 
+// M = 9..32 (plain GEMM): NB = 2..4 blocks of 8 lanes.  Each block's X
+// fragments and accumulators take registers, so the CTA runs fewer warps
+// (12 for two or three blocks, 8 for four), each with a deeper ring for the
+// same bytes in flight.
+constexpr int kStagesWide = 2;
+constexpr int wide_warps(int nb) { return nb <= 3 ? 12 : 8; }
+constexpr int wide_units_per_stage(int nb) { return nb <= 3 ? 8 : 12; }
+
 template <int M, int NW>
 struct KernelOf {
-    static constexpr int stages = NW == 1 ? kStagesPlain : kStagesFused;
-    static constexpr int ups = NW == 1 ? kUnitsPerStagePlain : kUnitsPerStageFused;
-    static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages, ups>; }
-    static size_t smem() { return (size_t)kWarps * stages * (NW * ups * kUnitBytes + 8) + kWarps * 8; }
+    static constexpr bool wide = M > kMaxM;
+    static constexpr int nb = (M + 7) / 8;
+    static constexpr int warps = wide ? wide_warps(nb) : kWarps;
+    static constexpr int stages = wide ? kStagesWide : NW == 1 ? kStagesPlain : kStagesFused;
+    static constexpr int ups = wide ? wide_units_per_stage(nb) : NW == 1 ? kUnitsPerStagePlain : kUnitsPerStageFused;
+    static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages, ups, warps>; }
+    static size_t smem() { return (size_t)warps * stages * (NW * ups * kUnitBytes + 8) + warps * 8; }
 };
 
 struct KernelInfo {
     void* fn = nullptr;
     size_t smem = 0;
+    int warps = 0;
     int blocks_per_sm = 0;  // filled on first use
 };
 
@@ -834,17 +877,28 @@ KernelInfo kernel_info_for(int M)
     case m:                                  \
         k.fn = KernelOf<m, NW>::fn();        \
         k.smem = KernelOf<m, NW>::smem();    \
+        k.warps = KernelOf<m, NW>::warps;    \
         break;
         NVFP4_CASE(1) NVFP4_CASE(2) NVFP4_CASE(3) NVFP4_CASE(4)
         NVFP4_CASE(5) NVFP4_CASE(6) NVFP4_CASE(7) NVFP4_CASE(8)
-#undef NVFP4_CASE
     }
+    if constexpr (NW == 1) {
+        switch (M) {
+            NVFP4_CASE(9) NVFP4_CASE(10) NVFP4_CASE(11) NVFP4_CASE(12)
+            NVFP4_CASE(13) NVFP4_CASE(14) NVFP4_CASE(15) NVFP4_CASE(16)
+            NVFP4_CASE(17) NVFP4_CASE(18) NVFP4_CASE(19) NVFP4_CASE(20)
+            NVFP4_CASE(21) NVFP4_CASE(22) NVFP4_CASE(23) NVFP4_CASE(24)
+            NVFP4_CASE(25) NVFP4_CASE(26) NVFP4_CASE(27) NVFP4_CASE(28)
+            NVFP4_CASE(29) NVFP4_CASE(30) NVFP4_CASE(31) NVFP4_CASE(32)
+        }
+    }
+#undef NVFP4_CASE
     return k;
 }
 
 std::mutex g_mu;
 DeviceState g_states[64];
-KernelInfo g_kernels[64][2][kMaxM];  // [device][kind][M-1]
+KernelInfo g_kernels[64][2][kWideMaxM];  // [device][kind][M-1]
 
 }  // namespace
 
@@ -893,14 +947,16 @@ int device_state(cudaStream_t stream, DeviceState** out)
 
 static int kernel_for(int dev, int kind, int M, KernelInfo** out)
 {
+    if (M < 1 || M > (kind == 0 ? kWideMaxM : kMaxM)) return NVFP4_ERR_M;
     std::lock_guard<std::mutex> lock(g_mu);
     KernelInfo& k = g_kernels[dev][kind][M - 1];
     if (k.blocks_per_sm == 0) {
         KernelInfo fresh = kind == 0 ? kernel_info_for<1>(M) : kernel_info_for<2>(M);
+        if (!fresh.fn) return NVFP4_ERR_M;
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(fresh.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)fresh.smem));
         int nb = 0;
-        NVFP4_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fresh.fn, kWarps * 32,
+        NVFP4_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fresh.fn, fresh.warps * 32,
                                                                      fresh.smem));
         if (nb < 1) return NVFP4_ERR_CUDA;
         fresh.blocks_per_sm = nb;
@@ -923,7 +979,8 @@ int validate_gemm(const GemmArgs& a)
     if (!a.X || !a.out) return NVFP4_ERR_ARG;
     for (int i = 0; i < nw; ++i)
         if (!a.wq[i] || !a.ws[i]) return NVFP4_ERR_ARG;
-    int st = check_m(a.M);
+    // the plain GEMM also takes M = 9..16 (two blocks of 8 lanes)
+    int st = a.kind == 0 ? ((a.M >= 1 && a.M <= kWideMaxM) ? NVFP4_OK : NVFP4_ERR_M) : check_m(a.M);
     if (st != NVFP4_OK) return st;
     st = check_shape(a.N, a.K);
     if (st != NVFP4_OK) return st;
@@ -939,13 +996,14 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
     int st = kernel_for(ds->device, a.kind, a.M, &k);
     if (st != NVFP4_OK) return st;
     const Geometry geo = geometry(a.N, a.K);
+    const int W = k->warps;
     long long ctas = (long long)ds->sm_count * k->blocks_per_sm;
-    const long long need = (geo.units + kWarps - 1) / kWarps;
+    const long long need = (geo.units + W - 1) / W;
     if (need < ctas) ctas = need;
-    if (ctas * kWarps > ds->max_warps) ctas = ds->max_warps / kWarps;
+    if (ctas * W > ds->max_warps) ctas = ds->max_warps / W;
     // Never more warps than units: every warp below total_warps gets a
     // non-empty range (the split-K combine relies on it).
-    const long long total_warps = ctas * kWarps < geo.units ? ctas * kWarps : geo.units;
+    const long long total_warps = ctas * W < geo.units ? ctas * W : geo.units;
 
     KParams p;
     const int nw = a.kind == 0 ? 1 : 2;
@@ -966,7 +1024,7 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ctas);
-    cfg.blockDim = dim3(kWarps * 32);
+    cfg.blockDim = dim3(W * 32);
     cfg.dynamicSmemBytes = k->smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1115,10 +1173,11 @@ int gemm_launch_warps(const GemmArgs& a, DeviceState* ds, long long* warps)
     int st = kernel_for(ds->device, a.kind, a.M, &k);
     if (st != NVFP4_OK) return st;
     const Geometry geo = geometry(a.N, a.K);
+    const int W = k->warps;
     long long ctas = (long long)ds->sm_count * k->blocks_per_sm;
-    const long long need = (geo.units + kWarps - 1) / kWarps;
+    const long long need = (geo.units + W - 1) / W;
     if (need < ctas) ctas = need;
-    *warps = ctas * kWarps;
+    *warps = ctas * W;
     return NVFP4_OK;
 }
 
@@ -1151,8 +1210,8 @@ using namespace nvfp4;
 extern "C" int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                                  float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream)
 {
-    // verify widths run on the tensor-memory kernel
-    if (M >= kVerifyMinM && M <= kVerifyMaxM) return launch_verify(X, M, wq_dev, ws_dev, gscale, Y, N, K, (cudaStream_t)stream);
+    // M = 17..64 run on the tensor-memory kernel; up to 16 on the register-MMA kernel
+    if (M > kWideMaxM && M <= kVerifyMaxM) return launch_verify(X, M, wq_dev, ws_dev, gscale, Y, N, K, (cudaStream_t)stream);
     GemmArgs a = {};
     a.kind = 0;
     a.X = X;

@@ -57,6 +57,7 @@ constexpr int kUnitQ = 1024;        // nibble bytes per unit
 constexpr int kUnitS = 128;         // scale bytes per unit
 constexpr int kUnitBytes = kUnitQ + kUnitS;
 constexpr int kMaxM = 8;            // decode lanes
+constexpr int kWideMaxM = 32;       // plain-GEMM rows on the register-MMA path (up to four blocks of 8)
 
 // bf16x2 bit positions of the two codes of a pair: sign, e1, e0, m.
 constexpr uint32_t kPairMask = 0x81C081C0u;

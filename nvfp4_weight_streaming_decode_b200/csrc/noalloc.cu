@@ -73,6 +73,7 @@ extern "C" int nvfp4_gemm_decode_noalloc(const void* X, int M, const uint8_t* wq
     a.out = Y;
     a.N = N;
     a.K = K;
+    if (M > kMaxM) return NVFP4_ERR_M;  // decode lanes only
     int st = validate_gemm(a);
     if (st != NVFP4_OK) return st;
     int dev = 0;

@@ -1,7 +1,8 @@
 """GPU parity of nvfp4_gemm_decode at verify widths, M = 9..64 (ignis README,
 "What sets it apart", "Speculative decoding (DFlash2)": lanes x (1 + drafts)
-rows verified in the same pass over the weights), which run on the
-tensor-memory (tcgen05) kernel, against the oracle."""
+rows verified in the same pass over the weights), against the oracle.  Widths
+9..16 run on the register-MMA decode kernel with two blocks of 8 lanes,
+17..64 on the tensor-memory (tcgen05) kernel."""
 import numpy as np
 import pytest
 import torch
@@ -23,7 +24,7 @@ def dev(cuda_device):
     return cuda_device
 
 
-@pytest.mark.parametrize("M", [9, 16, 17, 31, 33, 48, 63, 64])
+@pytest.mark.parametrize("M", [9, 10, 12, 15, 16, 17, 31, 33, 48, 63, 64])
 @pytest.mark.parametrize("N,K", [(32, 64), (256, 512), (300, 1040), (1000, 2048), (5120, 5120)])
 def test_verify_gemm_matches_oracle(dev, M, N, K):
     q, s = synth.matrix(50, N * 13 + K, N, K)
@@ -33,7 +34,7 @@ def test_verify_gemm_matches_oracle(dev, M, N, K):
     assert_gemm_close(Y, Yr, A, f"M={M} N={N} K={K}")
 
 
-@pytest.mark.parametrize("M", [9, 64])
+@pytest.mark.parametrize("M", [9, 16, 64])
 def test_verify_down_projection(dev, M):
     """K = 17,408 (the MLP down projection): long K ranges, many CTAs per tile pair."""
     N, K = 5120, 17408
@@ -44,7 +45,7 @@ def test_verify_down_projection(dev, M):
     assert_gemm_close(Y, Yr, A, f"down M={M}")
 
 
-@pytest.mark.parametrize("M", [16, 64])
+@pytest.mark.parametrize("M", [12, 16, 64])
 def test_verify_head_sampled(dev, M):
     """The vocabulary head (151,936 x 5,120, log-uniform scales) at a verify
     width, checked against the oracle on sampled rows."""
@@ -85,7 +86,7 @@ def test_verify_identity_is_exact(dev):
     for n in range(K):
         q[n, n // 2] |= 0x2 << (4 * (n % 2))
     s = np.full((K, K // 16), 0x38, np.uint8)
-    for M in (9, 24, 64):
+    for M in (9, 13, 16, 24, 64):
         X = synth.activations(synth.rng(53, M), M, K)
         Y = gemm_case(dev, q, s, X, gscale=1.0)
         assert np.array_equal(Y, (X.astype(np.uint32) << 16).view(np.float32)), M
@@ -93,3 +94,21 @@ def test_verify_identity_is_exact(dev):
 
 def test_verify_status_clean(dev):
     assert abi.nvfp4_device_status() == 0
+
+
+def test_wide_width_is_deterministic_and_matches_per_block_rows(dev):
+    """M = 13 on the register-MMA kernel: bit-identical across calls, and each
+    block of 8 lanes within the GEMM bound of the oracle (rows past M in the
+    second block feed only dropped columns)."""
+    N, K = 2048, 3072
+    q, s = synth.matrix(54, 0, N, K)
+    X = synth.activations(synth.rng(54, 1), 13, K)
+    wq, ws = packed(q, s, dev)
+    Xd = x_to_dev(X, dev)
+    Y1 = abi.gemm_decode(Xd, wq, ws, synth.GSCALE, N, K)
+    Y2 = abi.gemm_decode(Xd, wq, ws, synth.GSCALE, N, K)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int32), Y2.view(torch.int32))
+    Yr, A = oracle.gemm(X, q, s, synth.GSCALE)
+    assert_gemm_close(Y1[:8].cpu().numpy(), Yr[:8], A[:8], "lanes 0..7")
+    assert_gemm_close(Y1[8:].cpu().numpy(), Yr[8:], A[8:], "lanes 8..12")
