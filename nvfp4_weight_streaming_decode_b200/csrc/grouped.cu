@@ -119,7 +119,8 @@ __device__ void build_groups(const GParams& p, GroupTable& gt)
         const int e = p.route[tid];
         gt.exp[tid] = expert_ok(p, e) ? e : -1;
     }
-    __syncthreads();
+    // every thread sees the count of valid routes
+    const int nv = __syncthreads_count(tid < R && gt.exp[tid] >= 0);
     if (tid < R && gt.exp[tid] >= 0) {
         const int e = gt.exp[tid];
         int rank = 0, run = 0;  // position among valid routes; where this expert's run starts
@@ -133,21 +134,28 @@ __device__ void build_groups(const GParams& p, GroupTable& gt)
         gt.start[rank] = (rank - run) % 8 == 0 ? 1 : 0;
     }
     __syncthreads();
-    if (tid == 0) {
-        int nv = 0;
-        for (int q = 0; q < R; ++q) nv += gt.exp[q] >= 0 ? 1 : 0;
-        int g = -1;
-        for (int r = 0; r < nv; ++r) {
-            if (gt.start[r]) {
-                ++g;
-                gt.g_expert[g] = gt.exp[gt.sorted[r]];
-                gt.g_first[g] = r;
-                gt.g_rows[g] = 0;
-            }
-            ++gt.g_rows[g];
-        }
-        gt.n_groups = g + 1;
+    // Group index of each sorted position: the count of group starts up to it
+    // (a ballot prefix within each warp, then across the first four warps).
+    __shared__ int warp_starts[NVFP4_GROUPED_MAX_ROUTES / 32];
+    const bool st = tid < nv && gt.start[tid] != 0;
+    const unsigned ballot = __ballot_sync(0xffffffffu, st);
+    const int lane = tid & 31, w = tid >> 5;
+    if (w < NVFP4_GROUPED_MAX_ROUTES / 32 && lane == 0) warp_starts[w] = __popc(ballot);
+    __syncthreads();
+    if (st) {
+        int g = __popc(ballot & ((1u << lane) - 1u));
+        for (int k = 0; k < w; ++k) g += warp_starts[k];
+        gt.g_expert[g] = gt.exp[gt.sorted[tid]];
+        gt.g_first[g] = tid;
     }
+    if (tid == 0) {
+        int ng = 0;
+        for (int k = 0; k < NVFP4_GROUPED_MAX_ROUTES / 32; ++k) ng += warp_starts[k];
+        gt.n_groups = ng;
+    }
+    __syncthreads();
+    // a group runs to the next group's first position (or to the end)
+    if (tid < gt.n_groups) gt.g_rows[tid] = (tid + 1 < gt.n_groups ? gt.g_first[tid + 1] : nv) - gt.g_first[tid];
     __syncthreads();
 }
 
@@ -285,7 +293,7 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
                     float* dst = p.partials + ((size_t)gw * 2 + slot_id) * kGSlot + lane * 8;
                     reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
                     reinterpret_cast<float4*>(dst)[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
-                    __threadfence();
+                    // the lanes' stores are ordered before lane 0's release by the warp barrier
                     __syncwarp();
                     unsigned last = 0;
                     if (lane == 0) {
@@ -302,12 +310,27 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
                         for (int r = 0; r < 2; ++r)
     #pragma unroll
                             for (int k = 0; k < 4; ++k) acc[r][k] = 0.f;
-                        for (long long w = glo; w <= ghi; ++w) {
-                            const int ws = (w == glo) ? glo_slot : 0;
-                            const float4* src = reinterpret_cast<const float4*>(p.partials + ((size_t)w * 2 + ws) * kGSlot + lane * 8);
-                            const float4 a = __ldcg(src), b = __ldcg(src + 1);
-                            acc[0][0] += a.x; acc[0][1] += a.y; acc[0][2] += a.z; acc[0][3] += a.w;
-                            acc[1][0] += b.x; acc[1][1] += b.y; acc[1][2] += b.z; acc[1][3] += b.w;
+                        // four contributors' loads in flight at a time, added in warp order
+                        for (long long w0 = glo; w0 <= ghi; w0 += 4) {
+                            float4 pa[4], pb[4];
+#pragma unroll
+                            for (int b = 0; b < 4; ++b) {
+                                const long long w = w0 + b;
+                                if (w <= ghi) {
+                                    const int ws = (w == glo) ? glo_slot : 0;
+                                    const float4* src = reinterpret_cast<const float4*>(
+                                        p.partials + ((size_t)w * 2 + ws) * kGSlot + lane * 8);
+                                    pa[b] = __ldcg(src);
+                                    pb[b] = __ldcg(src + 1);
+                                }
+                            }
+#pragma unroll
+                            for (int b = 0; b < 4; ++b) {
+                                if (w0 + b <= ghi) {
+                                    acc[0][0] += pa[b].x; acc[0][1] += pa[b].y; acc[0][2] += pa[b].z; acc[0][3] += pa[b].w;
+                                    acc[1][0] += pb[b].x; acc[1][1] += pb[b].y; acc[1][2] += pb[b].z; acc[1][3] += pb[b].w;
+                                }
+                            }
                         }
                         if (lane == 0) p.counters[tg] = 0u;  // every contributor is in
                     }
