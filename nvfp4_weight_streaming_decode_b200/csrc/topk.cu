@@ -322,11 +322,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p)
     if (tid < p.k) {
         ck[tid] = tid < kl ? sh.out_key[tid] : 0u;
         ci[tid] = tid < kl ? sh.out_idx[tid] : kPadIdx - (uint32_t)(s * p.k + tid);
-        // each writer makes its stores visible at GPU scope before the count-in
-        __threadfence();
     }
-    // The count-in (thread 0, acquire/release) follows every writer's fence;
-    // its acquire side orders the merge's loads after the other CTAs' stores.
+    // The CTA barrier orders every writer's stores before thread 0's count-in,
+    // whose release side publishes them at GPU scope (cumulatively) and whose
+    // acquire side orders the merge's loads after the other CTAs' stores.
     __syncthreads();
     if (tid == 0) {
         unsigned old;
