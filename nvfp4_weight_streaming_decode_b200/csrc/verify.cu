@@ -1,4 +1,5 @@
-// verify.cu -- the decode GEMM at verify widths, M = 9..64 rows of X.
+// verify.cu -- the decode GEMM at verify widths, M = 33..64 rows of X (up to
+// 32 run on the decode kernel with several lane blocks).
 //
 // ignis README, "What sets it apart", "Speculative decoding (DFlash2)": each
 // lane's drafts are verified in the same pass over the weights, so the GEMM
@@ -8,17 +9,21 @@
 //     Y[m][n] = gscale * sum_k x[m][k] * e2m1(q[n][k]) * e4m3(s[n][k/16]).
 //
 // At these widths the product no longer fits the register MMA path, so the
-// multiply runs on the fifth-generation tensor cores (tcgen05) with the
-// accumulators in tensor memory:
+// multiply runs on the fifth-generation tensor cores (tcgen05) with both the
+// accumulators and the A operand in tensor memory:
 //   * A CTA (one per SM) owns a contiguous range of (512-row tile group,
 //     64-column chunk) units -- stream-K at CTA granularity -- so every SM
 //     gets the same number of weight bytes, whatever the shape.
 //   * Sixteen dequantisation warps each stream one 32-row tile of the group
 //     through their own ring of 1-D bulk copies, dequantise it exactly (the
 //     same bit placement and bf16 scale multiply as the M <= 8 kernel) and
-//     store it as bf16 into the MMA's K-major operand layout in shared
-//     memory; they also stage the chunk of X (the MMA's N side, M rows
-//     padded to a multiple of 16).  A and X are double-buffered.
+//     store it as bf16 into tensor memory with one tcgen05.st per row group:
+//     the 16x256b store shape takes the m16n8k16 A fragment as it stands,
+//     so the MMA's k order is the fragment's (per step s, k = 4t + j is the
+//     chunk's column 16t + 4s + j).  They also stage the chunk of X (the
+//     MMA's N side, M rows padded to a multiple of 16) in shared memory in
+//     that k order.  A and X are double-buffered; keeping A out of shared
+//     memory leaves its bandwidth to the weight ring and X.
 //   * One thread of a seventeenth warp issues tcgen05.mma (M = 128, N =
 //     16..64, K = 16; four per tile and chunk) into four accumulators in
 //     tensor memory and commits each chunk to an mbarrier that frees its
@@ -52,20 +57,24 @@ constexpr int kVWarps = 4 * kVTiles;           // dequantisation warps: one per 
 constexpr int kVCtasPerSM = 1;                 // one CTA per SM: shared memory holds its operands
 constexpr int kVBufs = 2;                      // operand (A, X) buffers: chunks in flight to the tensor cores
 constexpr int kVThreads = (kVWarps + 1) * 32;  // + the MMA / tensor-memory warp
-constexpr int kVStages = 3;                    // per-warp ring depth, one unit per stage
+constexpr int kVStages = 6;                    // per-warp ring depth, one unit per stage
 constexpr int kVTileRows = 128;                // MMA M
 constexpr int kVMaxNL = 64;                    // MMA N at most (M rows of X, padded to 16)
-constexpr int kABytes = kVTileRows * kChunkK * 2;  // one tile's bf16 A for one chunk: 16 KB
 constexpr int kXBytes = kVMaxNL * kChunkK * 2;     // one chunk of X: 8 KB
+// Tensor memory (512 columns): accumulators in columns [0, 4 * nl) (nl <= 64),
+// the bf16 A operand from column 256: per buffer and tile, 128 lanes x 32
+// columns (a chunk's 64 values per row, two per column).
+constexpr int kVTmemCols = 512;
+constexpr int kATmemCol = kVTiles * kVMaxNL;       // 256
+constexpr int kATmemTileCols = kChunkK / 2;        // 32
 constexpr int kVGroupRows = kVTiles * kVTileRows;  // 512
 constexpr int kVSlotFloats = kVMaxNL * kVGroupRows;  // a partial: [512 rows][64 m] floats
 constexpr int kVMaxGroups = 1 << 16;                // tile groups a call may have
 constexpr int kVMaxSplit = 4;                      // CTAs per tile group at most, on average
 
 // shared-memory map (bytes)
-constexpr int kOffA = 0;                                   // [2 buffers][kVTiles tiles][16 KB]
-constexpr int kOffX = kOffA + kVBufs * kVTiles * kABytes;  // [kVBufs buffers][8 KB]
-constexpr int kOffRing = kOffX + kVBufs * kXBytes;         // [kVWarps warps][3 stages][1152 B]
+constexpr int kOffX = 0;                                   // [kVBufs buffers][8 KB]
+constexpr int kOffRing = kOffX + kVBufs * kXBytes;         // [kVWarps warps][kVStages stages][1152 B]
 constexpr int kOffBar = kOffRing + kVWarps * kVStages * kUnitBytes;
 // barriers: ring[8][3], full[2], empty[2], acc, acc_free, part_done, last_ready, fin
 constexpr int kBarRing = 0, kBarFull = kVWarps * kVStages, kBarEmpty = kBarFull + kVBufs, kBarAcc = kBarEmpty + kVBufs,
@@ -112,22 +121,36 @@ __device__ __forceinline__ uint32_t kmajor_off(int row, int octet)
     return (uint32_t)((row >> 3) * 1024 + octet * 128 + (row & 7) * 16);
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w)
+__device__ __forceinline__ void st_shared_v2(uint32_t a, uint32_t x, uint32_t y)
 {
-    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+    asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
+
+// 16 lanes x 4 x 256 bits of this warp's lane quarter from registers: register
+// 4i + j goes to lane (taddr's lane) + (t / 4) + 8 * (j / 2), column (taddr's
+// column) + 8i + 2 * (t % 4) + (j % 2), for thread t -- the layout of the
+// m16n8k16 A fragment, so a lane's dequantised words go out as they are.
+__device__ __forceinline__ void tc_st_16x256b_x4(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] . B[smem]^T, bf16 x bf16 -> f32, no output lane disabled.
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate)
+// D[tmem] (+)= A[tmem] . B[smem]^T, bf16 x bf16 -> f32, no output lane disabled.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
 {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
         : "memory");
 }
 
@@ -205,7 +228,7 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kVWarps) {
-        // tensor memory for the two accumulators (a power of two >= 32 columns)
+        // tensor memory for the accumulators and the A operand (all 512 columns)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(base + kOffMisc),
                      "r"(p.tmem_cols)
                      : "memory");
@@ -263,12 +286,25 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                     xr[h] = *reinterpret_cast<const uint4*>(p.X + nrow * p.K + col);
             }
         };
+        // X in the MMA's k order: step s takes, as k = 4u + j (u = 0..3, j = 0..3),
+        // the chunk's columns 16u + 4s + j -- the order in which the dequantised
+        // words go to tensor memory.  Each 8-byte half of a 16-byte piece (four
+        // columns) lands in step s's octet u / 2, at byte 8 * (u % 2).
         auto store_x = [&](int bb, const uint4 (&xr)[2]) {
             const uint32_t xb = base + kOffX + bb * kXBytes;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int pc = w * 32 + lane + h * kVWarps * 32;
-                if (pc < p.NL * 8) st_shared_v4(xb + kmajor_off(pc >> 3, pc & 7), xr[h].x, xr[h].y, xr[h].z, xr[h].w);
+                if (pc < p.NL * 8) {
+                    const int nrow = pc >> 3, o = pc & 7;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int c0 = 8 * o + 4 * half;  // first of the four columns
+                        const int u = c0 >> 4, st = (c0 >> 2) & 3;
+                        st_shared_v2(xb + kmajor_off(nrow, 2 * st + (u >> 1)) + 8 * (u & 1),
+                                     half ? xr[h].z : xr[h].x, half ? xr[h].w : xr[h].y);
+                    }
+                }
             }
         };
         // X of the first chunk goes straight into buffer 0; every later chunk's X is
@@ -277,7 +313,6 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
         uint4 xr[2];
         load_x(c0, xr);
         store_x(0, xr);
-        const int g = lane >> 2, t = lane & 3;
         const int trow = 32 * (w & 3);  // first row of this warp in its 128-row tile
         const int tt = w >> 2;          // which tile of the group
         int seg = 0, split = 0;
@@ -306,8 +341,12 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                 q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
             }
             const int b = j % kVBufs;  // buffer b is free: the previous iteration's end waited for it
-            // A: this warp's 32 rows of its tile for this chunk, bf16, K-major core matrices
-            const uint32_t abuf = base + kOffA + (b * kVTiles + tt) * kABytes;
+            // A: this warp's 32 rows of its tile for this chunk, bf16, into tensor memory
+            // (lanes = rows, two values per column).  Word s of row group r holds rows
+            // 16r+g (a[s][0], a[s][2]) and 16r+g+8 (a[s][1], a[s][3]) at columns
+            // 16t+4s+{0,1} and {2,3}: MMA step s, k = 4t + {0,1} and {2,3}, i.e. the
+            // step's columns 2t and 2t + 1.
+            const uint32_t acol = tmem + (uint32_t)(kATmemCol + (b * kVTiles + tt) * kATmemTileCols);
             uint32_t S[2][2] = {{0u, 0u}, {0u, 0u}};
             if (valid) scale_pairs(sw, S);
 #pragma unroll
@@ -321,13 +360,13 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                         a[s][0] = a[s][1] = a[s][2] = a[s][3] = 0u;
                     }
                 }
-                const int row_lo = trow + 16 * r + g, row_hi = row_lo + 8;
-                // a[s][0]/a[s][2]: row_lo, columns 16t+4s+{0,1} / {2,3}; a[s][1]/a[s][3]: row_hi
-                st_shared_v4(abuf + kmajor_off(row_lo, 2 * t), a[0][0], a[0][2], a[1][0], a[1][2]);
-                st_shared_v4(abuf + kmajor_off(row_lo, 2 * t + 1), a[2][0], a[2][2], a[3][0], a[3][2]);
-                st_shared_v4(abuf + kmajor_off(row_hi, 2 * t), a[0][1], a[0][3], a[1][1], a[1][3]);
-                st_shared_v4(abuf + kmajor_off(row_hi, 2 * t + 1), a[2][1], a[2][3], a[3][1], a[3][3]);
+                const uint32_t v[16] = {a[0][0], a[0][2], a[0][1], a[0][3], a[1][0], a[1][2], a[1][1], a[1][3],
+                                        a[2][0], a[2][2], a[2][1], a[2][3], a[3][0], a[3][2], a[3][1], a[3][3]};
+                tc_st_16x256b_x4(acol + ((uint32_t)(trow + 16 * r) << 16), v);
             }
+            // the A stores are complete before the MMA thread is told
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
             // The tensor cores read A and X, and the next bulk copy writes this ring
             // slot, through the async proxy: order this warp's shared-memory accesses
             // first.  The slot is refilled only now, after the dequantisation above
@@ -444,6 +483,8 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                     pend_hi = (j + 1 + kVStages < n) ? j + 1 + kVStages : n;
                     break;
                 }
+                // the MMAs that read this buffer's A (tensor memory) are done: later stores follow them
+                tc_fence_after();
                 store_x(b1, xr);
             }
             if (++c == (int)KC) {
@@ -476,11 +517,11 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                 const uint32_t xs = base + kOffX + b * kXBytes;
 #pragma unroll
                 for (int tt = 0; tt < kVTiles; ++tt) {
-                    const uint32_t as = base + kOffA + (b * kVTiles + tt) * kABytes;
+                    const uint32_t at = tmem + (uint32_t)(kATmemCol + (b * kVTiles + tt) * kATmemTileCols);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc_mma(tmem + (uint32_t)(tt * p.NL), kmajor_desc(as + 256 * kk), kmajor_desc(xs + 256 * kk),
-                               p.idesc, (first && kk == 0) ? 0u : 1u);
+                        tc_mma_ts(tmem + (uint32_t)(tt * p.NL), at + (uint32_t)(8 * kk), kmajor_desc(xs + 256 * kk),
+                                  p.idesc, (first && kk == 0) ? 0u : 1u);
                 }
                 any = true;
                 tc_commit(bars + 8 * (kBarEmpty + b));
@@ -579,9 +620,7 @@ int verify_geometry(int M, int64_t N, int64_t K, int sm_count, VerifyGeometry* g
     if (ctas > g->units) ctas = g->units;
     g->ctas = ctas;
     g->nl = (M + 15) / 16 * 16;
-    int cols = 32;
-    while (cols < kVTiles * g->nl) cols *= 2;
-    g->tmem_cols = cols;
+    g->tmem_cols = kVTmemCols;  // accumulators (4 x nl <= 256 columns) and the double-buffered A operand
     return NVFP4_OK;
 }
 
