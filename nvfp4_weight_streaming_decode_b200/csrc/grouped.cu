@@ -37,6 +37,7 @@ __device__ unsigned int g_grouped_status;
 namespace {
 
 constexpr int kGWarps = 16;     // one CTA of 16 warps per SM
+static_assert(kGWarps * 32 >= 4 * NVFP4_GROUPED_MAX_ROUTES, "grouping counts each route with four threads");
 constexpr int kGStages = 3;     // per-warp ring depth
 constexpr int kGUPS = 4;        // units per stage (a stage crossing to the next expert takes one copy per part)
 constexpr int kGStage = kGUPS * kUnitBytes;
@@ -121,17 +122,29 @@ __device__ void build_groups(const GParams& p, GroupTable& gt)
     }
     // every thread sees the count of valid routes
     const int nv = __syncthreads_count(tid < R && gt.exp[tid] >= 0);
-    if (tid < R && gt.exp[tid] >= 0) {
-        const int e = gt.exp[tid];
-        int rank = 0, run = 0;  // position among valid routes; where this expert's run starts
-        for (int q = 0; q < R; ++q) {
-            const int eq = gt.exp[q];
-            if (eq < 0) continue;
-            if (eq < e || (eq == e && q < tid)) ++rank;
-            if (eq < e) ++run;
+    // Route r's rank among the valid routes (by expert, then position) and where its
+    // expert's run starts, counted by the four threads 4r..4r+3 over every fourth route
+    // and summed across the quad.
+    {
+        const int r = tid >> 2, part = tid & 3;
+        const int e = r < R ? gt.exp[r] : -1;
+        int rank = 0, run = 0;
+        if (e >= 0) {
+            for (int q = part; q < R; q += 4) {
+                const int eq = gt.exp[q];
+                if (eq < 0) continue;
+                if (eq < e || (eq == e && q < r)) ++rank;
+                if (eq < e) ++run;
+            }
         }
-        gt.sorted[rank] = tid;
-        gt.start[rank] = (rank - run) % 8 == 0 ? 1 : 0;
+        rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+        run += __shfl_xor_sync(0xffffffffu, run, 1);
+        rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+        run += __shfl_xor_sync(0xffffffffu, run, 2);
+        if (e >= 0 && part == 0) {
+            gt.sorted[rank] = r;
+            gt.start[rank] = (rank - run) % 8 == 0 ? 1 : 0;
+        }
     }
     __syncthreads();
     // Group index of each sorted position: the count of group starts up to it
