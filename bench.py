@@ -52,6 +52,9 @@ def parse_args():
                     help="only three direct calls of one workload GEMM at --width (for an ncu capture)")
     ap.add_argument("--topk-case", type=int, default=None,
                     help="only three top-k calls with this k over --width rows of 151,936 logits (for an ncu capture)")
+    ap.add_argument("--grouped-case", action="store_true",
+                    help="only three grouped expert calls (512 experts of 768 x 2,048, --width lanes, 10 picks each; "
+                         "for an ncu capture)")
     return ap.parse_args()
 
 
@@ -516,6 +519,30 @@ def run_gemm_case(args):
     return 0
 
 
+def run_grouped_case(args):
+    """Three nvfp4_gemm_grouped calls: 512 seeded experts of 768 x 2,048, --width lanes with 10 picks
+    each (three different seeded route tables)."""
+    import numpy as np
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi, build, synth
+    from nvfp4_weight_streaming_decode_b200.workloads import make_matrix
+    build.build()
+    dev = torch.device("cuda", 0)
+    E, T, N, K, M = 512, 10, 768, 2048, args.width
+    m = make_matrix(5, 0, E * N, K, dev)
+    qb, sb = (N // 32) * (K // 64) * 1024, (N // 32) * (K // 64) * 128
+    table = abi.expert_table([(m.wq[e * qb:(e + 1) * qb], m.ws[e * sb:(e + 1) * sb], synth.GSCALE)
+                              for e in range(E)], dev)
+    rng = np.random.default_rng(7)
+    X = synth.torch_activations(5, 2, M, K, dev)
+    for _ in range(3):
+        r = torch.from_numpy(np.stack([rng.choice(E, T, replace=False) for _ in range(M)]).astype(np.int32)).to(dev)
+        abi.gemm_grouped(X, r, table, E, N, K)
+    torch.cuda.synchronize()
+    print(json.dumps({"grouped_case": True, "M": M, "T": T, "E": E, "N": N, "K": K, "ok": True}))
+
+
 def run_topk_case(args):
     """Three nvfp4_topk calls over [--width][151,936] seeded N(0,1) logits."""
     import torch
@@ -691,6 +718,8 @@ def main():
         return run_gemm_case(args)
     if args.topk_case:
         return run_topk_case(args)
+    if args.grouped_case:
+        return run_grouped_case(args)
     return run_ours(args)
 
 
