@@ -840,6 +840,11 @@ namespace {
 // Two deep stages: the same bytes in flight per warp as three shallower ones,
 // in fewer, larger bulk copies (measured faster on the round at every width).
 constexpr int kStagesPlain = 2, kUnitsPerStagePlain = 6;
+// Plain GEMMs at M = 5..8 with few units per warp (a layer's projections, not
+// the head): three stages of 4 units, the same bytes in flight in smaller
+// copies, so a warp starts on its first units sooner.
+constexpr int kStagesPlainShort = 3, kUnitsPerStagePlainShort = 4;
+constexpr int kShortMinM = 5, kShortMaxUnitsPerWarp = 32;
 constexpr int kStagesFused = 2, kUnitsPerStageFused = 3;
 
 // M = 9..32 (plain GEMM): NB = 2..4 blocks of 8 lanes.  Each block's X
@@ -850,13 +855,14 @@ constexpr int kStagesWide = 2;
 constexpr int wide_warps(int nb) { return nb <= 3 ? 12 : 8; }
 constexpr int wide_units_per_stage(int nb) { return nb <= 3 ? 8 : 12; }
 
-template <int M, int NW>
+template <int M, int NW, bool SHORT = false>
 struct KernelOf {
     static constexpr bool wide = M > kMaxM;
     static constexpr int nb = (M + 7) / 8;
     static constexpr int warps = wide ? wide_warps(nb) : kWarps;
-    static constexpr int stages = wide ? kStagesWide : NW == 1 ? kStagesPlain : kStagesFused;
-    static constexpr int ups = wide ? wide_units_per_stage(nb) : NW == 1 ? kUnitsPerStagePlain : kUnitsPerStageFused;
+    static constexpr int stages = wide ? kStagesWide : NW == 2 ? kStagesFused : SHORT ? kStagesPlainShort : kStagesPlain;
+    static constexpr int ups = wide ? wide_units_per_stage(nb)
+                               : NW == 2 ? kUnitsPerStageFused : SHORT ? kUnitsPerStagePlainShort : kUnitsPerStagePlain;
     static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages, ups, warps>; }
     static size_t smem() { return (size_t)warps * stages * (NW * ups * kUnitBytes + 8) + warps * 8; }
 };
@@ -869,9 +875,24 @@ struct KernelInfo {
 };
 
 template <int NW>
-KernelInfo kernel_info_for(int M)
+KernelInfo kernel_info_for(int M, bool short_stages)
 {
     KernelInfo k;
+    if constexpr (NW == 1) {
+        if (short_stages) {
+            switch (M) {
+#define NVFP4_SHORT(m)                                     \
+    case m:                                                \
+        k.fn = KernelOf<m, 1, true>::fn();                 \
+        k.smem = KernelOf<m, 1, true>::smem();             \
+        k.warps = KernelOf<m, 1, true>::warps;             \
+        return k;
+                NVFP4_SHORT(5) NVFP4_SHORT(6) NVFP4_SHORT(7) NVFP4_SHORT(8)
+#undef NVFP4_SHORT
+            }
+            return k;
+        }
+    }
     switch (M) {
 #define NVFP4_CASE(m)                        \
     case m:                                  \
@@ -898,7 +919,7 @@ KernelInfo kernel_info_for(int M)
 
 std::mutex g_mu;
 DeviceState g_states[64];
-KernelInfo g_kernels[64][2][kWideMaxM];  // [device][kind][M-1]
+KernelInfo g_kernels[64][2][kWideMaxM][2];  // [device][kind][M-1][short stages]
 
 }  // namespace
 
@@ -945,13 +966,20 @@ int device_state(cudaStream_t stream, DeviceState** out)
     return NVFP4_OK;
 }
 
-static int kernel_for(int dev, int kind, int M, KernelInfo** out)
+// Whether a plain GEMM of this width and shape takes the short-stage kernel.
+static bool short_stages(int kind, int M, long long units, const DeviceState* ds)
+{
+    return kind == 0 && M >= kShortMinM && M <= kMaxM &&
+           units < (long long)kShortMaxUnitsPerWarp * ds->sm_count * kWarps;
+}
+
+static int kernel_for(int dev, int kind, int M, bool shrt, KernelInfo** out)
 {
     if (M < 1 || M > (kind == 0 ? kWideMaxM : kMaxM)) return NVFP4_ERR_M;
     std::lock_guard<std::mutex> lock(g_mu);
-    KernelInfo& k = g_kernels[dev][kind][M - 1];
+    KernelInfo& k = g_kernels[dev][kind][M - 1][shrt ? 1 : 0];
     if (k.blocks_per_sm == 0) {
-        KernelInfo fresh = kind == 0 ? kernel_info_for<1>(M) : kernel_info_for<2>(M);
+        KernelInfo fresh = kind == 0 ? kernel_info_for<1>(M, shrt) : kernel_info_for<2>(M, false);
         if (!fresh.fn) return NVFP4_ERR_M;
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(fresh.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)fresh.smem));
@@ -969,7 +997,9 @@ static int kernel_for(int dev, int kind, int M, KernelInfo** out)
 int prepare_kernel(DeviceState* ds, int kind, int M)
 {
     KernelInfo* k = nullptr;
-    return kernel_for(ds->device, kind, M, &k);
+    int st = kernel_for(ds->device, kind, M, false, &k);
+    if (st == NVFP4_OK && kind == 0 && M >= kShortMinM && M <= kMaxM) st = kernel_for(ds->device, kind, M, true, &k);
+    return st;
 }
 
 int validate_gemm(const GemmArgs& a)
@@ -992,10 +1022,10 @@ int validate_gemm(const GemmArgs& a)
 
 int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* ds)
 {
-    KernelInfo* k = nullptr;
-    int st = kernel_for(ds->device, a.kind, a.M, &k);
-    if (st != NVFP4_OK) return st;
     const Geometry geo = geometry(a.N, a.K);
+    KernelInfo* k = nullptr;
+    int st = kernel_for(ds->device, a.kind, a.M, short_stages(a.kind, a.M, geo.units, ds), &k);
+    if (st != NVFP4_OK) return st;
     const int W = k->warps;
     long long ctas = (long long)ds->sm_count * k->blocks_per_sm;
     const long long need = (geo.units + W - 1) / W;
@@ -1169,10 +1199,10 @@ int round_persistent_launch(void* params_host, unsigned* d_arrive, int M, int gr
 
 int gemm_launch_warps(const GemmArgs& a, DeviceState* ds, long long* warps)
 {
-    KernelInfo* k = nullptr;
-    int st = kernel_for(ds->device, a.kind, a.M, &k);
-    if (st != NVFP4_OK) return st;
     const Geometry geo = geometry(a.N, a.K);
+    KernelInfo* k = nullptr;
+    int st = kernel_for(ds->device, a.kind, a.M, short_stages(a.kind, a.M, geo.units, ds), &k);
+    if (st != NVFP4_OK) return st;
     const int W = k->warps;
     long long ctas = (long long)ds->sm_count * k->blocks_per_sm;
     const long long need = (geo.units + W - 1) / W;
