@@ -24,7 +24,7 @@ def dev(cuda_device):
     return cuda_device
 
 
-@pytest.mark.parametrize("M", [9, 10, 12, 15, 16, 17, 31, 33, 48, 63, 64])
+@pytest.mark.parametrize("M", [9, 10, 12, 15, 16, 17, 24, 25, 31, 32, 33, 48, 63, 64])
 @pytest.mark.parametrize("N,K", [(32, 64), (256, 512), (300, 1040), (1000, 2048), (5120, 5120)])
 def test_verify_gemm_matches_oracle(dev, M, N, K):
     q, s = synth.matrix(50, N * 13 + K, N, K)
