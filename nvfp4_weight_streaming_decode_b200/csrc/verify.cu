@@ -61,6 +61,7 @@ constexpr int kVStages = 6;                    // per-warp ring depth, one unit 
 constexpr int kVTileRows = 128;                // MMA M
 constexpr int kVMaxNL = 64;                    // MMA N at most (M rows of X, padded to 16)
 constexpr int kXBytes = kVMaxNL * kChunkK * 2;     // one chunk of X: 8 KB
+static_assert(kVMaxNL * 8 <= kVWarps * 32, "each dequantisation thread stages at most one 16-byte piece of X");
 // Tensor memory (512 columns): accumulators in columns [0, 4 * nl) (nl <= 64),
 // the bf16 A operand from column 256: per buffer and tile, 128 lanes x 32
 // columns (a chunk's 64 values per row, two per column).
@@ -274,43 +275,41 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
         // X and the outputs come from / go to the previous kernel's buffers
         asm volatile("griddepcontrol.wait;" ::: "memory");
 
-        // X pieces of this lane (16 bytes each; at most two per lane as nl <= 64)
-        auto load_x = [&](int cc, uint4 (&xr)[2]) {
+        // X pieces of this thread: piece pc = 16 bytes of row pc / 8, columns 8 (pc % 8)
+        // .. +7 of a chunk (nl <= 64 rows: at most one piece per thread, 512 threads).
+        // In the MMA's k order step s takes, as k = 4u + j (u = 0..3, j = 0..3), the
+        // chunk's columns 16u + 4s + j -- the order in which the dequantised words go
+        // to tensor memory -- so each 8-byte half of a piece (four columns) lands in
+        // step s's octet u / 2, at byte 8 * (u % 2).  Everything but the chunk's column
+        // and the buffer is fixed per thread, so it is worked out once here.
+        const int pc = w * 32 + lane;
+        const bool x_piece = pc < p.NL * 8;                  // this thread stages a piece
+        const int x_row = pc >> 3, x_o = pc & 7;
+        const bool x_row_ok = x_piece && x_row < p.M;        // rows past M stay zero
+        const uint16_t* x_src = p.X + (long long)(x_row_ok ? x_row : 0) * p.K + 8 * x_o;
+        uint32_t x_dst[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int pc = w * 32 + lane + h * kVWarps * 32;
-                xr[h] = make_uint4(0u, 0u, 0u, 0u);
-                const int nrow = pc >> 3, o = pc & 7;
-                const long long col = (long long)cc * kChunkK + 8 * o;
-                if (pc < p.NL * 8 && nrow < p.M && col < p.K)
-                    xr[h] = *reinterpret_cast<const uint4*>(p.X + nrow * p.K + col);
-            }
+        for (int half = 0; half < 2; ++half) {
+            const int c4 = 8 * x_o + 4 * half;  // first of the four columns
+            const int u = c4 >> 4, st = (c4 >> 2) & 3;
+            x_dst[half] = kmajor_off(x_piece ? x_row : 0, 2 * st + (u >> 1)) + 8 * (u & 1);
+        }
+        auto load_x = [&](int cc, uint4& xr) {
+            xr = make_uint4(0u, 0u, 0u, 0u);
+            if (x_row_ok && (long long)cc * kChunkK + 8 * x_o < p.K)
+                xr = *reinterpret_cast<const uint4*>(x_src + (long long)cc * kChunkK);
         };
-        // X in the MMA's k order: step s takes, as k = 4u + j (u = 0..3, j = 0..3),
-        // the chunk's columns 16u + 4s + j -- the order in which the dequantised
-        // words go to tensor memory.  Each 8-byte half of a 16-byte piece (four
-        // columns) lands in step s's octet u / 2, at byte 8 * (u % 2).
-        auto store_x = [&](int bb, const uint4 (&xr)[2]) {
-            const uint32_t xb = base + kOffX + bb * kXBytes;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int pc = w * 32 + lane + h * kVWarps * 32;
-                if (pc < p.NL * 8) {
-                    const int nrow = pc >> 3, o = pc & 7;
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int c0 = 8 * o + 4 * half;  // first of the four columns
-                        const int u = c0 >> 4, st = (c0 >> 2) & 3;
-                        st_shared_v2(xb + kmajor_off(nrow, 2 * st + (u >> 1)) + 8 * (u & 1),
-                                     half ? xr[h].z : xr[h].x, half ? xr[h].w : xr[h].y);
-                    }
-                }
+        auto store_x = [&](int bb, const uint4& xr) {
+            if (x_piece) {
+                const uint32_t xb = base + kOffX + bb * kXBytes;
+                st_shared_v2(xb + x_dst[0], xr.x, xr.y);
+                st_shared_v2(xb + x_dst[1], xr.z, xr.w);
             }
         };
         // X of the first chunk goes straight into buffer 0; every later chunk's X is
         // loaded at the top of the iteration before it and stored at that iteration's
         // end, once its buffer is free (the loads have landed by then).
-        uint4 xr[2];
+        uint4 xr;
         load_x(c0, xr);
         store_x(0, xr);
         const int trow = 32 * (w & 3);  // first row of this warp in its 128-row tile
