@@ -63,6 +63,14 @@ def test_argument_errors_return_before_any_cuda_call(lib):
     assert abi.nvfp4_gemm_decode(p + 8, 1, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ALIGN
     assert abi.nvfp4_gemm_decode(p, 1, p + 4, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ALIGN
     assert abi.nvfp4_gemm_decode(p, 1, p, p, 1.0, p + 2, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    # widths 9..32 take the decode kernel's validation (lane blocks), 33..64 the tcgen05 kernel's
+    assert abi.nvfp4_gemm_decode(p, 16, p, p, 1.0, p + 4, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_decode(p, 32, p + 8, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_gemm_decode(p, 24, p, p, 1.0, p, 32, 0, None) == abi.NVFP4_ERR_SHAPE
+    # the no-allocation entry point takes decode lanes only
+    assert abi.nvfp4_gemm_decode_noalloc(p, 0, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_gemm_decode_noalloc(p, 9, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
+    assert abi.nvfp4_gemm_decode_noalloc(p, 16, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
     assert abi.nvfp4_gemm_gateup_silu(p, 1, p, p, 1.0, None, p, 1.0, p, 32, 64, None) == \
         abi.NVFP4_ERR_ARG
     assert abi.nvfp4_gemm_gateup_silu(p, 10, p, p, 1.0, p, p, 1.0, p, 32, 64, None) == abi.NVFP4_ERR_M
