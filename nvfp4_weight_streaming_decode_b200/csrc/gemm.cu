@@ -259,26 +259,40 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
             if (lane == 0) atomicOr(&g_device_status, 4u);
             warp_wait(gather_bar, 0u);
         }
-        for (int c = 0; c < nb; ++c) {
-            float4 x[NA * 2];
-            if (gathered) {
-                const uint32_t src = gather_smem + c * kPartBytes + lane * (NA * 32);
+        // with one accumulator set, two contributors' loads in flight at a time (more
+        // registers here would make the callers save theirs); added in warp order
+        constexpr int kPair = NA == 1 ? 2 : 1;
+        for (int c = 0; c < nb; c += kPair) {
+            float4 x[kPair][NA * 2];
+            const int cnt = nb - c < kPair ? nb - c : kPair;
 #pragma unroll
-                for (int k = 0; k < NA * 2; ++k)
-                    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                                 : "=f"(x[k].x), "=f"(x[k].y), "=f"(x[k].z), "=f"(x[k].w)
-                                 : "r"(src + 16 * k));
-            } else {
-                const long long w = glo + c;
-                const int ws = (w == glo) ? glo_slot : 0;
-                load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), x);
+            for (int e = 0; e < kPair; ++e) {
+                if (e < cnt) {
+                    if (gathered) {
+                        const uint32_t src = gather_smem + (c + e) * kPartBytes + lane * (NA * 32);
+#pragma unroll
+                        for (int k = 0; k < NA * 2; ++k)
+                            asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                         : "=f"(x[e][k].x), "=f"(x[e][k].y), "=f"(x[e][k].z), "=f"(x[e][k].w)
+                                         : "r"(src + 16 * k));
+                    } else {
+                        const long long w = glo + c + e;
+                        const int ws = (w == glo) ? glo_slot : 0;
+                        load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), x[e]);
+                    }
+                }
             }
 #pragma unroll
-            for (int k = 0; k < NA * 2; ++k) {
-                sum[k >> 1][k & 1][0] += x[k].x;
-                sum[k >> 1][k & 1][1] += x[k].y;
-                sum[k >> 1][k & 1][2] += x[k].z;
-                sum[k >> 1][k & 1][3] += x[k].w;
+            for (int e = 0; e < kPair; ++e) {
+                if (e < cnt) {
+#pragma unroll
+                    for (int k = 0; k < NA * 2; ++k) {
+                        sum[k >> 1][k & 1][0] += x[e][k].x;
+                        sum[k >> 1][k & 1][1] += x[e][k].y;
+                        sum[k >> 1][k & 1][2] += x[e][k].z;
+                        sum[k >> 1][k & 1][3] += x[e][k].w;
+                    }
+                }
             }
         }
     }
