@@ -17,6 +17,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -68,11 +69,19 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_code(text):
+    """Source text without comments and blank lines: what the compiler sees of it."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_hash():
+    """Hash of the decode GEMM's sources, comments aside (a comment edit does not change the kernel)."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "nvfp4_weight_streaming_decode_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "nvfp4_weight_streaming_decode_b200", "csrc", name)) as f:
+            h.update(kernel_code(f.read()).encode())
     return h.hexdigest()[:16]
 
 

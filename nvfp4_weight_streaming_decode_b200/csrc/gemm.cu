@@ -326,8 +326,8 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
 
 // STAGES shared-memory stages per warp, each holding UPS consecutive units of
 // each of the NW matrices (one bulk copy per plane and matrix per stage).
-// W warps per CTA (one CTA per SM).  M up to 16: lanes 8..15 form a second
-// block of the MMA's 8-wide side, sharing every dequantised word.
+// W warps per CTA (one CTA per SM).  M up to 32: lanes 8b..8b+7 form block b
+// of the MMA's 8-wide side, and every dequantised word feeds each block.
 template <int M, int NW, int STAGES, int UPS, int W>
 __global__ void __launch_bounds__(W * 32, kMinBlocks)
 decode_gemm_kernel(const KParams p)
@@ -1023,7 +1023,7 @@ int validate_gemm(const GemmArgs& a)
     if (!a.X || !a.out) return NVFP4_ERR_ARG;
     for (int i = 0; i < nw; ++i)
         if (!a.wq[i] || !a.ws[i]) return NVFP4_ERR_ARG;
-    // the plain GEMM also takes M = 9..16 (two blocks of 8 lanes)
+    // the plain GEMM also takes M = 9..32 (two to four blocks of 8 lanes)
     int st = a.kind == 0 ? ((a.M >= 1 && a.M <= kWideMaxM) ? NVFP4_OK : NVFP4_ERR_M) : check_m(a.M);
     if (st != NVFP4_OK) return st;
     st = check_shape(a.N, a.K);

@@ -4,7 +4,7 @@
 // ignis README, "What sets it apart", "Speculative decoding (DFlash2)": each
 // lane's drafts are verified in the same pass over the weights, so the GEMM
 // takes lanes x (1 + drafts) rows of X -- up to 8 x 8 = 64.  The format and
-// the result are those of the M <= 8 kernel (ignis, "Models and artifacts",
+// the result are those of the decode kernel (ignis, "Models and artifacts",
 // "The artifact": 4-bit floating point with one scale per 16 values):
 //     Y[m][n] = gscale * sum_k x[m][k] * e2m1(q[n][k]) * e4m3(s[n][k/16]).
 //
@@ -16,7 +16,7 @@
 //     gets the same number of weight bytes, whatever the shape.
 //   * Sixteen dequantisation warps each stream one 32-row tile of the group
 //     through their own ring of 1-D bulk copies, dequantise it exactly (the
-//     same bit placement and bf16 scale multiply as the M <= 8 kernel) and
+//     same bit placement and bf16 scale multiply as the decode kernel) and
 //     store it as bf16 into tensor memory with one tcgen05.st per row group:
 //     the 16x256b store shape takes the m16n8k16 A fragment as it stands,
 //     so the MMA's k order is the fragment's (per step s, k = 4t + j is the

@@ -1,8 +1,8 @@
 """GPU parity of nvfp4_gemm_decode at verify widths, M = 9..64 (ignis README,
 "What sets it apart", "Speculative decoding (DFlash2)": lanes x (1 + drafts)
 rows verified in the same pass over the weights), against the oracle.  Widths
-9..16 run on the register-MMA decode kernel with two blocks of 8 lanes,
-17..64 on the tensor-memory (tcgen05) kernel."""
+9..32 run on the register-MMA decode kernel with two to four blocks of 8
+lanes, 33..64 on the tensor-memory (tcgen05) kernel."""
 import numpy as np
 import pytest
 import torch
