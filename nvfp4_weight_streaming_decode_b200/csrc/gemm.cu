@@ -406,8 +406,11 @@ decode_gemm_kernel(const KParams p)
     // MMA output columns m >= M, which depend on nothing else and which the
     // epilogue drops, and every lane then runs the same unpredicated loads.
     const uint16_t* xp = p.X + (long long)(g % M) * p.K + chunk * kChunkK + 16 * t;
-    // the second block's row, (8 + g) % M, as an offset from the first's
-    const long long x_delta = NB > 1 ? (long long)((8 + g) % M - g % M) * p.K : 0;
+    // block b's row, (8b + g) % M (a valid row: only the last block reaches past
+    // M, and by less than M), as an offset from block 0's
+    long long x_off[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) x_off[b] = (long long)((8 * b + g) % M - g % M) * p.K;
     int col = chunk * kChunkK + 16 * t;                 // this lane's first column in the unit
     const uint32_t q_off = 16 * lane, s_off = 4 * lane;
     int slot = 0;
@@ -441,7 +444,7 @@ decode_gemm_kernel(const KParams p)
 #pragma unroll
             for (int v = 0; v < UPS; ++v) {
 #pragma unroll
-                for (int b = 0; b < NB; ++b) ld_x32_keep(xp + b * x_delta + v * kChunkK, true, xf[b]);
+                for (int b = 0; b < NB; ++b) ld_x32_keep(xp + x_off[b] + v * kChunkK, true, xf[b]);
                 const uint8_t* sq = stage + v * kUnitQ + q_off;
                 const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
 #pragma unroll
@@ -460,7 +463,7 @@ decode_gemm_kernel(const KParams p)
                 // This lane's 16 columns of X (zeros past K).
                 uint32_t xw[NB][8];
 #pragma unroll
-                for (int b = 0; b < NB; ++b) ld_x32(xp + b * x_delta, col < K32, xw[b]);
+                for (int b = 0; b < NB; ++b) ld_x32(xp + x_off[b], col < K32, xw[b]);
                 const uint8_t* sq = stage + v * kUnitQ + q_off;
                 const uint8_t* ss = stage + UPS * kUnitQ + v * kUnitS + s_off;
 #pragma unroll
