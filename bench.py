@@ -461,6 +461,51 @@ def grouped_sweep(dev, hbm_peak):
     return {"kernel": "grouped_kernel", "cases": out}
 
 
+def percentile(xs, q):
+    """q-th percentile of a list, linear between closest ranks (numpy's default)."""
+    ys = sorted(xs)
+    if not ys:
+        return None
+    pos = (len(ys) - 1) * q / 100.0
+    lo = int(pos)
+    hi = min(lo + 1, len(ys) - 1)
+    return ys[lo] + (ys[hi] - ys[lo]) * (pos - lo)
+
+
+def stream_read_peak(dev, stream, hbm_peak, gib=4, reps=10):
+    """Read-only HBM bandwidth with the library's own probe (nvfp4_stream_read):
+    one pass over a `gib` GiB buffer per launch, four CTAs per SM, best and
+    median of `reps` launches under CUDA events.  A second denominator beside
+    the measured copy peak; the roofline keeps the copy figure."""
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi
+    nbytes = gib << 30
+    buf = torch.zeros(nbytes // 4, dtype=torch.int32, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ctas = 4 * sms
+    out = torch.empty((ctas,), dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            abi.stream_read(buf, ctas, out, stream)
+    times = []
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            abi.stream_read(buf, ctas, out, stream)
+            e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    del buf, out
+    torch.cuda.empty_cache()
+    best = nbytes / min(times) / 1e9
+    return {"gbs": best, "median_gbs": nbytes / statistics.median(times) / 1e9, "bytes": nbytes, "ctas": ctas,
+            "reps": reps, "of_copy_peak": best / hbm_peak,
+            "kernel": "stream_read_kernel (nvfp4_stream_read: 16-byte cache-streaming loads, XOR per CTA)"}
+
+
 def topk_detail(logits, dev, hbm_peak):
     """Device time of nvfp4_topk on the round's own head logits (FP32
     [8][151,936]), for rows 1 and 8 and k = 1, 8, 64: 50 calls captured in a
@@ -598,21 +643,27 @@ def run_ours(args):
             rnd.replay(M, stream)
     torch.cuda.synchronize()
 
-    # per-width round times (detail): 20 replays each
-    by_width = {}
+    # per-width round times (detail): 20 replays each, an event after every replay
+    # for the median and p90 beside the mean
+    by_width, p50_by_width, p90_by_width = {}, {}, {}
     if args.profile:
         args.no_sweep = args.no_cpu_baseline = True
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_rep = 20
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_rep + 1)]
     for m in (range(1, 9) if not args.profile else ()):
         with torch.cuda.stream(stream):
             for _ in range(3):
                 rnd.replay(m, stream)
-            e0.record(stream)
-            for _ in range(20):
+            evs[0].record(stream)
+            for j in range(n_rep):
                 rnd.replay(m, stream)
-            e1.record(stream)
-        e1.synchronize()
-        by_width[m] = e0.elapsed_time(e1) / 20
+                evs[j + 1].record(stream)
+        evs[-1].synchronize()
+        per = [evs[j].elapsed_time(evs[j + 1]) for j in range(n_rep)]
+        by_width[m] = evs[0].elapsed_time(evs[-1]) / n_rep
+        p50_by_width[m] = statistics.median(per)
+        p90_by_width[m] = percentile(per, 90)
 
     # the timed region: K replays at width M
     clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
@@ -665,6 +716,10 @@ def run_ours(args):
                 "kernel": ("round_kernel (persistent round, one launch per round)" if args.round_mode == "persistent"
                            else "decode_gemm_kernel (one launch per round node)")}
 
+    read_peak = None
+    if rank == 0 and not args.no_sweep:
+        read_peak = stream_read_peak(dev, stream, hbm_peak)
+
     topk = None
     if rank == 0 and not args.no_sweep:
         rnd.replay(8, stream)
@@ -701,6 +756,10 @@ def run_ours(args):
             "round_ms_by_width": by_width,
             "round_GBps_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 for m, t in by_width.items()},
             "round_frac_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 / hbm_peak for m, t in by_width.items()},
+            "round_ms_p50_by_width": p50_by_width,
+            "round_ms_p90_by_width": p90_by_width,
+            "read_peak": read_peak,
+            "round_frac_of_read_peak": (value / read_peak["gbs"]) if read_peak else None,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_host.numel() * 2,

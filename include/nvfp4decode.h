@@ -325,6 +325,22 @@ NVFP4_API int nvfp4_gemm_grouped(const void* X, int x_per_route, const int32_t* 
 NVFP4_API int nvfp4_verify_geometry(int M, int64_t N, int64_t K, int sm_count, int64_t* ctas, int64_t* units,
                                     int* nl);
 
+/*
+ * Measurement aid: read `bytes` of device memory once, as the decode round's
+ * weight stream does (README, "The decode round": the round is weight
+ * streaming at the card's bandwidth), to measure the read-only HBM bandwidth
+ * that the round's GB/s is compared with beside the copy figure.
+ *
+ * buf: device, 16-byte aligned, `bytes` a positive multiple of 16; it is only
+ * read.  out: device u32[ctas], 4-byte aligned; CTA c writes out[c], the XOR
+ * of the 32-bit words it read, so the XOR over all of `out` equals the XOR of
+ * every 32-bit word of `buf`.  ctas: grid size, 1..2^20 (four per SM keeps
+ * enough loads in flight for the full bandwidth).  One asynchronous launch.
+ * Returns NVFP4_ERR_ARG (NULL pointer, ctas out of range), NVFP4_ERR_SHAPE,
+ * NVFP4_ERR_ALIGN or NVFP4_ERR_CUDA (launch failed).
+ */
+NVFP4_API int nvfp4_stream_read(const void* buf, size_t bytes, uint32_t* out, int ctas, nvfp4_stream_t stream);
+
 /* Text for a status code (static storage). */
 NVFP4_API const char* nvfp4_status_string(int status);
 

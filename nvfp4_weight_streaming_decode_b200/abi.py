@@ -76,6 +76,7 @@ _SIGNATURES = {
     "nvfp4_unpack_debug": (_I, [_P, _P, _I64, _I64, _P, _P, _P]),
     "nvfp4_host_dequant_unit": (_I, [_P, _P, _F, _P]),
     "nvfp4_host_pack_unit": (_I, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
+    "nvfp4_stream_read": (_I, [_P, _SZ, _P, _I, _P]),
     "nvfp4_status_string": (ctypes.c_char_p, [_I]),
     "nvfp4_last_cuda_error": (_I, []),
     "nvfp4_device_status": (_I, []),
@@ -236,6 +237,10 @@ def nvfp4_host_pack_unit(wq_canon, ws_canon, N, K, tile, chunk, q_unit, s_unit):
                                        q_unit, s_unit)
 
 
+def nvfp4_stream_read(buf, nbytes, out, ctas, stream):
+    return load().nvfp4_stream_read(buf, int(nbytes), out, int(ctas), _s(stream))
+
+
 def nvfp4_status_string(status):
     return status_string(status)
 
@@ -336,6 +341,19 @@ def topk(logits, k, V=None, values=None, indices=None, stream=None):
     check(nvfp4_topk(logits.data_ptr(), rows, V, logits.stride(0), k, values.data_ptr(), indices.data_ptr(),
                      _stream_ptr(stream)), "nvfp4_topk")
     return values, indices
+
+
+def stream_read(buf, ctas, out=None, stream=None):
+    """Read every byte of the contiguous device tensor `buf` once (nvfp4_stream_read);
+    returns the uint32 [ctas] device tensor of per-CTA XORs (as int32)."""
+    import torch
+    if not buf.is_contiguous():
+        raise ValueError("buf must be contiguous")
+    if out is None:
+        out = torch.empty((ctas,), dtype=torch.int32, device=buf.device)
+    check(nvfp4_stream_read(buf.data_ptr(), buf.numel() * buf.element_size(), out.data_ptr(), ctas,
+                            _stream_ptr(stream)), "nvfp4_stream_read")
+    return out
 
 
 def dequant_debug(wq, ws, gscale, N, K, stream=None):

@@ -1,8 +1,11 @@
 """Host-side helpers of bench.py (no GPU): the kernel-source hash that ties the
 committed DRAM-traffic summary to the decode GEMM's code ignores comments and
-blank lines, and nothing else."""
+blank lines, and nothing else; the percentile used for the per-replay round
+times agrees with numpy's."""
 import os
 import sys
+
+import pytest
 
 sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 
@@ -24,3 +27,10 @@ def test_kernel_code_keeps_code_changes_visible():
 def test_kernel_hash_is_stable():
     h = bench.kernel_hash()
     assert len(h) == 16 and h == bench.kernel_hash()
+
+
+@pytest.mark.parametrize("xs", [[1.0], [2.0, 1.0], [float(i) for i in range(20)], [0.3, 5.1, 4.9, 5.0, 7.2, 5.05]])
+@pytest.mark.parametrize("q", [0, 50, 90, 100])
+def test_percentile_matches_numpy(xs, q):
+    import numpy as np
+    assert bench.percentile(xs, q) == pytest.approx(float(np.percentile(xs, q)), rel=1e-12, abs=1e-12)

@@ -107,6 +107,15 @@ def test_argument_errors_return_before_any_cuda_call(lib):
     assert abi.nvfp4_topk(p + 4, 1, 100, 100, 1, p, p, None) == abi.NVFP4_ERR_ALIGN
     assert abi.nvfp4_topk(p, 1, 100, 102, 1, p, p, None) == abi.NVFP4_ERR_ALIGN
     assert abi.nvfp4_topk(p, 1, 100, 100, 1, p + 2, p, None) == abi.NVFP4_ERR_ALIGN
+    # read-only stream probe
+    assert abi.nvfp4_stream_read(None, 64, p, 4, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_stream_read(p, 64, None, 4, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_stream_read(p, 64, p, 0, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_stream_read(p, 64, p, (1 << 20) + 1, None) == abi.NVFP4_ERR_ARG
+    assert abi.nvfp4_stream_read(p, 0, p, 4, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_stream_read(p, 72, p, 4, None) == abi.NVFP4_ERR_SHAPE
+    assert abi.nvfp4_stream_read(p + 8, 64, p, 4, None) == abi.NVFP4_ERR_ALIGN
+    assert abi.nvfp4_stream_read(p, 64, p + 2, 4, None) == abi.NVFP4_ERR_ALIGN
 
 
 @pytest.mark.parametrize("rows", [1, 2, 3, 8, 13, 64])
