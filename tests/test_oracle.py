@@ -173,6 +173,31 @@ def test_gemm_brute_force_against_numpy_matmul():
                                rtol=1e-12, atol=1e-15)
 
 
+@pytest.mark.parametrize("M", [9, 16, 17, 33, 64])
+def test_gemm_brute_force_at_verify_widths(M):
+    # the verify widths (lanes x (1 + drafts), up to 64 rows) use the same oracle
+    for (N, K) in [(5, 32), (33, 208)]:
+        g = synth.rng(300 + M, N * 1000 + K)
+        q = synth.codes(g, N, K)
+        s = synth.scales(g, N, K)
+        X = synth.activations(g, M, K)
+        Y, A = oracle.gemm(X, q, s, 1.0 / 64)
+        Wd = _dense_weights(q, s)
+        Xf = _bf16_to_f64(X)
+        assert np.allclose(Y, (Xf @ Wd.T) / 64, rtol=1e-12, atol=1e-12), (M, N, K)
+        rows = np.array([N - 1, 0, N // 2])
+        Yr, Ar = oracle.gemm_rows(X, q, s, 1.0 / 64, rows)
+        assert np.array_equal(Yr, Y[:, rows]) and np.array_equal(Ar, A[:, rows])
+
+
+def test_gemm_identity_weights_at_64_rows():
+    K = 128
+    q, s = _identity_planes(K)
+    X = synth.activations(synth.rng(12, 12), 64, K)
+    Y, _ = oracle.gemm(X, q, s, 1.0)
+    assert np.array_equal(Y, _bf16_to_f64(X))
+
+
 @pytest.mark.parametrize("c,sb", [(0x2, 0x38), (0x7, 0x7E), (0xB, 0x30), (0x1, 0x01), (0x0, 0x40)])
 def test_gemm_constant_code_closed_form(c, sb):
     M, N, K = 3, 5, 160
