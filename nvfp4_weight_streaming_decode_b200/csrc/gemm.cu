@@ -61,15 +61,6 @@ struct KParams {
     unsigned* counters;
 };
 
-__device__ __forceinline__ uint4 ld_nc_v4(const void* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 // 32 bytes of X into x when `pred`; x keeps its contents otherwise.
 __device__ __forceinline__ void ld_x32_keep(const void* p, bool pred, uint32_t (&x)[8])
 {
@@ -164,8 +155,6 @@ __device__ __forceinline__ void load_partial(const float* src, float4 (&v)[NW * 
 #pragma unroll
     for (int k = 0; k < NW * 2; ++k) v[k] = ld_cg_f4(src + 4 * k);
 }
-
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // End of a tile for this warp, after it stored its sums in its partial slot.
 // A tile the warp covered alone goes straight to the epilogue.  Otherwise the
