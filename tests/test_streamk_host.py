@@ -3,7 +3,8 @@ every unit is owned by exactly one warp, the owner formula inverts the range
 formula, each partial tile's contributors are counted right, and no two
 partial tiles share a counter or a partial-sum slot.  These are the integer
 formulas of the kernel (range_begin / range_owner / slot choice), replayed
-in Python over many grid sizes."""
+in Python over many grid sizes.  Also the X row each lane block loads at
+widths 1..32: always a row of X, and the lane's own row where it has one."""
 import itertools
 
 import pytest
@@ -46,3 +47,23 @@ def test_stream_k_assignment(n_tiles, k_chunks, TW):
             assert key not in slots, "two partial tiles share a slot"
             slots[key] = tile
             assert w < TW and slot in (0, 1)
+
+
+def x_row(M, g, b):
+    """Row of X that lane group g of lane block b loads in the decode kernel:
+    block 0's row g % M plus the block's offset ((8b + g) % M - g % M)."""
+    return g % M + ((8 * b + g) % M - g % M)
+
+
+@pytest.mark.parametrize("M", range(1, 33))
+def test_lane_block_x_rows_stay_inside_x(M):
+    # NB = ceil(M / 8) blocks of 8 lanes; a lane whose row 8b + g is a real
+    # row reads exactly that row, and every other lane reads some row of X
+    # (its MMA column is dropped), never one past the last
+    NB = -(-M // 8)
+    for b in range(NB):
+        for g in range(8):
+            r = x_row(M, g, b)
+            assert 0 <= r < M, (M, g, b, r)
+            if 8 * b + g < M:
+                assert r == 8 * b + g
