@@ -2,6 +2,7 @@
 model of the device layout against the oracle.  No GPU and no kernel launch:
 every call here returns before the library touches CUDA."""
 import ctypes
+import os
 
 import numpy as np
 import pytest
@@ -213,3 +214,20 @@ def test_verify_geometry_rejects():
     assert abi.nvfp4_verify_geometry(65, 32, 64, 148)[0] == abi.NVFP4_ERR_M
     assert abi.nvfp4_verify_geometry(16, 32, 40, 148)[0] == abi.NVFP4_ERR_SHAPE
     assert abi.nvfp4_verify_geometry(16, 0, 64, 148)[0] == abi.NVFP4_ERR_SHAPE
+
+
+def test_header_compiles_as_c99_and_links_from_c(lib, tmp_path):
+    """include/nvfp4decode.h is a C header: a C99 program built with -Wall
+    -Wextra -Werror against it links the library and gets the expected answers
+    from its host-side calls (tests/abi_c_check.c)."""
+    import subprocess
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    libdir = os.path.dirname(abi.LIB_PATH)
+    exe = str(tmp_path / "abi_c_check")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(root, "include"),
+                    os.path.join(here, "abi_c_check.c"), "-o", exe, "-L", libdir, "-lnvfp4decode",
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
