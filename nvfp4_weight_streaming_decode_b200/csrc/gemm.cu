@@ -4,7 +4,9 @@
 // README, "The decode round": all lanes share one pass over the weights,
 // which streams at the card's memory bandwidth), and the fused gate/up
 // variant H = bf16(silu(Xg) * Xu) that reads both projections in the same
-// pass.
+// pass.  The same kernel takes verify widths M = 9..32 (README, "What sets
+// it apart", "Speculative decoding (DFlash2)") as two to four blocks of 8
+// lanes, each dequantised word feeding one MMA per block.
 //
 // Work split ("stream-K"): the matrix is a sequence of 32 x 64 units stored
 // contiguously in tile-major order.  Every warp of the grid takes one
@@ -18,7 +20,9 @@
 // contributors arrives last: each writes its partial sums to the workspace,
 // bumps the tile's counter, and the last one adds the partials in warp order
 // (fixed, so results are bit-identical run to run) and runs the epilogue.
-// No thread ever waits on another warp or CTA.
+// In the plain and fused kernels no thread ever waits on another warp or
+// CTA; the persistent round kernel at the end of the file is the one place
+// where the grid meets, at a bounded barrier between nodes.
 //
 // PDL: every kernel signals its dependents at entry, issues its weight
 // copies (which depend on nothing), and only then waits for the preceding
@@ -39,7 +43,8 @@ namespace nvfp4 {
 
 __device__ unsigned int g_device_status;
 
-constexpr int kWarps = 16;                 // warps per CTA: one CTA per SM, so every warp has equal priority
+constexpr int kWarps = 16;                 // warps per CTA at M <= 8 (one CTA per SM, every warp at equal priority);
+                                           // the lane-block kernels run 12 or 8 (wide_warps below)
 constexpr int kMinBlocks = 1;              // CTAs per SM the register budget is sized for
 constexpr int kSlotFloats = 512;           // partial-sum slot: 2 matrices x 32 rows x 8 lanes
 
