@@ -229,6 +229,32 @@ def oracle_sample(device, seconds_budget):
                                    f"of the round's layer-0 q/k/v matrix, K={hidden}, {elapsed:.1f} s")
 
 
+def round_weight_bytes(layers, hidden, ffn, vocab):
+    """Weight bytes one round streams: every matrix in 32 x 64 units of 1,024 code bytes and
+    128 scale bytes (q/k/v stacked, o, gate, up and down per layer, then the head)."""
+    def mat(N, K):
+        return -(-N // 32) * -(-K // 64) * (1024 + 128)
+    per_layer = mat(3 * hidden, hidden) + mat(hidden, hidden) + 2 * mat(ffn, hidden) + mat(hidden, ffn)
+    return layers * per_layer + mat(vocab, hidden)
+
+
+def round_config(args, world, weight_bytes, nodes, graph_nodes):
+    """The bench line's config: the same dict for both arms."""
+    w = round_workload()
+    return {"workload": "round_64layers_head_m1to8", "width_M": args.width, "layers": args.layers,
+            "hidden": w["hidden"], "ffn": w["ffn"], "vocab": w["vocab"],
+            "weight_bytes_per_round": weight_bytes, "gemm_nodes": nodes,
+            "graph_nodes": graph_nodes, "round_mode": args.round_mode,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (13.8 GB of weights per round)"}
+
+
+def round_workload():
+    """Dimensions of the 64-layer round (hidden, ffn, vocab)."""
+    from nvfp4_weight_streaming_decode_b200 import synth
+    return synth.WORKLOADS[4]
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -238,7 +264,8 @@ def run_reference(args):
 
     import oracle
     from nvfp4_weight_streaming_decode_b200 import synth
-    hidden = synth.WORKLOADS[4]["hidden"]
+    w4 = synth.WORKLOADS[4]
+    hidden = w4["hidden"]
     q_full, s_full = synth.matrix(4, 0, 3 * hidden, hidden)
     Xb = synth.activations(synth.rng(4, 0), args.width, hidden)
     per_step_rows = 2048
@@ -263,8 +290,9 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / max(1, len(times)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "round_64layers_head_m1to8 (sampled rows, CPU oracle)",
-                   "width_M": args.width, "hidden": hidden},
+        "config": round_config(args, world, round_weight_bytes(args.layers, hidden, w4["ffn"], w4["vocab"]),
+                               4 * args.layers + 1,
+                               4 * args.layers + 1 if args.round_mode == "chain" else None),
         "cpu_baseline": {"value": gbs, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": gbs, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -746,12 +774,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random NVFP4 codes/scales, N(0,1) bf16 activations)",
-            "config": {"workload": "round_64layers_head_m1to8", "width_M": M, "layers": args.layers,
-                       "hidden": w["hidden"], "ffn": w["ffn"], "vocab": w["vocab"],
-                       "weight_bytes_per_round": weight_bytes, "gemm_nodes": nodes,
-                       "graph_nodes": graph_nodes, "round_mode": args.round_mode,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (13.8 GB of weights per round)"},
+            "config": round_config(args, world, weight_bytes, nodes, graph_nodes),
             "round_ms": ms_per_step,
             "round_ms_by_width": by_width,
             "round_GBps_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 for m, t in by_width.items()},

@@ -34,3 +34,21 @@ def test_kernel_hash_is_stable():
 def test_percentile_matches_numpy(xs, q):
     import numpy as np
     assert bench.percentile(xs, q) == pytest.approx(float(np.percentile(xs, q)), rel=1e-12, abs=1e-12)
+
+
+def test_round_weight_bytes_of_the_64_layer_round():
+    # 64 x (q/k/v 15,360 x 5,120 + o 5,120^2 + gate and up 17,408 x 5,120 + down 5,120 x 17,408)
+    # + head 151,936 x 5,120, at 0.5625 bytes per weight (all sizes are whole 32 x 64 units)
+    elems = 64 * (4 * 5120 * 5120 + 3 * 17408 * 5120) + 151936 * 5120
+    assert bench.round_weight_bytes(64, 5120, 17408, 151936) == elems * 9 // 16 == 13_838_376_960
+    # a ragged shape pads to whole units
+    assert bench.round_weight_bytes(0, 5120, 17408, 33) == 2 * 80 * 1152
+
+
+def test_reference_arm_config_equals_the_gpu_arm_config():
+    import argparse
+    args = argparse.Namespace(width=8, layers=64, round_mode="chain")
+    a = bench.round_config(args, 1, bench.round_weight_bytes(64, 5120, 17408, 151936), 257, 257)
+    assert a["workload"] == "round_64layers_head_m1to8" and a["weight_bytes_per_round"] == 13_838_376_960
+    assert a["gemm_nodes"] == a["graph_nodes"] == 257 and a["parallelism"] == "single GPU"
+    assert bench.round_config(args, 4, 1, 257, 257)["parallelism"] == "replicas x4"
