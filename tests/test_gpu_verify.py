@@ -34,7 +34,7 @@ def test_verify_gemm_matches_oracle(dev, M, N, K):
     assert_gemm_close(Y, Yr, A, f"M={M} N={N} K={K}")
 
 
-@pytest.mark.parametrize("M", [9, 16, 64])
+@pytest.mark.parametrize("M", [9, 16, 24, 31, 64])
 def test_verify_down_projection(dev, M):
     """K = 17,408 (the MLP down projection): long K ranges, many CTAs per tile pair."""
     N, K = 5120, 17408
@@ -45,7 +45,7 @@ def test_verify_down_projection(dev, M):
     assert_gemm_close(Y, Yr, A, f"down M={M}")
 
 
-@pytest.mark.parametrize("M", [12, 16, 64])
+@pytest.mark.parametrize("M", [12, 16, 25, 64])
 def test_verify_head_sampled(dev, M):
     """The vocabulary head (151,936 x 5,120, log-uniform scales) at a verify
     width, checked against the oracle on sampled rows."""
