@@ -349,8 +349,18 @@ NVFP4_API int nvfp4_last_cuda_error(void);
 
 /*
  * Device-side status of the current device: 0 when every kernel finished its
- * bounded waits, else a nonzero code.  Reading it synchronises the device;
- * a nonzero status also clears the flag and re-zeroes the split-K counters.
+ * bounded waits, else an OR of these flags:
+ *    1  decode GEMM: a warp's bulk-copy ring wait gave up
+ *    2  persistent round: the grid barrier between nodes gave up
+ *    4  decode GEMM: the split-K gather's copy wait gave up (sums then read
+ *       from global memory)
+ *    8  verify widths (33..64): a streaming warp's wait gave up
+ *   16  verify widths (33..64): the MMA thread's wait gave up
+ *   32  grouped experts: a route named an expert outside 0..E-1 or with
+ *       misaligned planes (its rows are zero)
+ *   64  grouped experts: a bounded wait gave up
+ * Reading it synchronises the device; a nonzero status also clears the flags
+ * and re-zeroes the split-K counters.
  */
 NVFP4_API int nvfp4_device_status(void);
 

@@ -1251,7 +1251,7 @@ using namespace nvfp4;
 extern "C" int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                                  float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream)
 {
-    // M = 17..64 run on the tensor-memory kernel; up to 16 on the register-MMA kernel
+    // M = 33..64 run on the tensor-memory kernel; up to 32 on the register-MMA kernel (lane blocks past 8)
     if (M > kWideMaxM && M <= kVerifyMaxM) return launch_verify(X, M, wq_dev, ws_dev, gscale, Y, N, K, (cudaStream_t)stream);
     GemmArgs a = {};
     a.kind = 0;
