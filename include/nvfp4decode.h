@@ -126,9 +126,10 @@ NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, con
  * that loads the library holds it until the process exits.
  *
  * Arguments, layout and result are those of nvfp4_gemm_decode at M = 1..8
- * (the same kernel runs); verify widths are not taken here (NVFP4_ERR_M).  The first call on a device resolves the array's device
- * address (cudaGetSymbolAddress) with that device current, so make that first
- * call before any stream capture.  Each call clears the arrival counters on
+ * (the same kernel runs); verify widths are not taken here (NVFP4_ERR_M).
+ * The first call on a device resolves the array's device address
+ * (cudaGetSymbolAddress) with that device current, so make that first call
+ * before any stream capture.  Each call clears the arrival counters on
  * `stream` before the kernel.  All calls share the one array, which keeps the
  * previous call's contents: calls that overlap on the GPU (other streams,
  * other host threads) race on it and must be serialised by the caller.
