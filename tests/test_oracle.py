@@ -1,9 +1,10 @@
 """Pins of the float64 oracle against facts that do not come from the oracle.
 
 Sources of truth used here: the E2M1 value list of the standard element
-format (tests/golden/e2m1_values.txt), torch's float8_e4m3fn decoder (a
-library routine), scipy's expit, numpy's matmul and sum, a hand-worked
-example (tests/golden/worked_example.txt), and closed forms that hold for
+format (tests/golden/e2m1_values.txt), torch's float8_e4m3fn decoder and
+ml_dtypes' float4_e2m1fn / float8_e4m3fn decoders (library routines),
+scipy's expit, numpy's matmul and sum, a hand-worked example
+(tests/golden/worked_example.txt), and closed forms that hold for
 structured weights.  Each would fail for a plausible mistake in the oracle:
 a wrong bias or subnormal rule (tables), swapped nibbles or a wrong scale
 index (probes, worked example), a dropped scale or global scale (closed
@@ -83,6 +84,19 @@ def test_e4m3_table_matches_torch_float8():
     assert sorted(np.nonzero(nan)[0].tolist()) == [0x7F, 0xFF]
     assert np.array_equal(e4[~nan], ref[~nan])
     assert np.array_equal(np.signbit(e4[~nan]), np.signbit(ref[~nan]))
+
+
+def test_tables_match_ml_dtypes():
+    # a second library decoder for both formats (ml_dtypes' float4_e2m1fn and
+    # float8_e4m3fn, one code per byte), independent of the golden list and torch
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    e2, e4 = oracle.tables()
+    ref2 = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(e2, ref2) and np.array_equal(np.signbit(e2), np.signbit(ref2))
+    ref4 = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    nan = np.isnan(ref4)
+    assert np.array_equal(np.isnan(e4), nan)
+    assert np.array_equal(e4[~nan], ref4[~nan]) and np.array_equal(np.signbit(e4[~nan]), np.signbit(ref4[~nan]))
 
 
 def test_table_invariants():
