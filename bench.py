@@ -746,7 +746,11 @@ def run_ours(args):
 
     read_peak = None
     if rank == 0 and not args.no_sweep:
-        read_peak = stream_read_peak(dev, stream, hbm_peak)
+        try:
+            read_peak = stream_read_peak(dev, stream, hbm_peak)
+        except (RuntimeError, MemoryError) as e:  # context only: never lose the bench line to it
+            torch.cuda.synchronize()
+            read_peak = {"gbs": None, "error": str(e)[:200]}
 
     topk = None
     if rank == 0 and not args.no_sweep:
@@ -782,7 +786,7 @@ def run_ours(args):
             "round_ms_p50_by_width": p50_by_width,
             "round_ms_p90_by_width": p90_by_width,
             "read_peak": read_peak,
-            "round_frac_of_read_peak": (value / read_peak["gbs"]) if read_peak else None,
+            "round_frac_of_read_peak": (value / read_peak["gbs"]) if read_peak and read_peak["gbs"] else None,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_host.numel() * 2,
