@@ -129,12 +129,15 @@ NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, con
  * (the same kernel runs); verify widths are not taken here (NVFP4_ERR_M).
  * The first call on a device resolves the array's device address
  * (cudaGetSymbolAddress) with that device current, so make that first call
- * before any stream capture.  Each call clears the arrival counters on
+ * before any stream capture (a first call made while `stream` is captured
+ * returns NVFP4_ERR_CAPTURE).  Each call clears the arrival counters on
  * `stream` before the kernel.  All calls share the one array, which keeps the
  * previous call's contents: calls that overlap on the GPU (other streams,
  * other host threads) race on it and must be serialised by the caller.
- * Returns NVFP4_ERR_SCRATCH if the launch would need more warps than the array
- * holds (a device with more than 160 SMs).
+ * A launch that would use more warps than the array holds (a device with more
+ * than 160 SMs) runs with 2,560 warps instead; the result is the same GEMM
+ * within the bound, though not bit-identical to nvfp4_gemm_decode on such a
+ * device, whose work split differs.
  */
 NVFP4_API int nvfp4_gemm_decode_noalloc(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                                         float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);
@@ -145,7 +148,10 @@ NVFP4_API int nvfp4_gemm_decode_noalloc(const void* X, int M, const uint8_t* wq_
  *   H[m][n] = bf16( silu(g) * u ),  silu(g) = g / (1 + exp(-g)).
  * X bf16 [M][K]; H bf16 [M][Nff]; the gate and up matrices are separate
  * Nff x K matrices in device layout.  Same workspace rules as
- * nvfp4_gemm_decode.
+ * nvfp4_gemm_decode.  The pages describe no such fused projection: the 27B
+ * body has an MLP in every layer ("Models and artifacts", model table), and
+ * fusing its gate and up projections with the SiLU-multiply into one pass over
+ * both weight matrices is this library's design.
  */
 NVFP4_API int nvfp4_gemm_gateup_silu(const void* X, int M,
                            const uint8_t* wq_gate, const uint8_t* ws_gate, float gscale_gate,

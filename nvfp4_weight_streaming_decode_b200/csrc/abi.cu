@@ -43,7 +43,7 @@ extern "C" const char* nvfp4_status_string(int status)
     switch (status) {
     case NVFP4_OK: return "ok";
     case NVFP4_ERR_ARG: return "invalid argument (NULL pointer, bad kind or count)";
-    case NVFP4_ERR_M: return "M must be in 1..8";
+    case NVFP4_ERR_M: return "M out of range for this entry point (1..8; nvfp4_gemm_decode also takes 9..64)";
     case NVFP4_ERR_SHAPE: return "bad shape: need N >= 1, K >= 16, K % 16 == 0";
     case NVFP4_ERR_ALIGN: return "device pointer not 16-byte aligned";
     case NVFP4_ERR_BAD_SCALE: return "scale plane holds an E4M3 NaN code (0x7F or 0xFF)";

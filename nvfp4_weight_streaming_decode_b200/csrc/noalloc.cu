@@ -35,11 +35,16 @@ NoAllocDevice g_noalloc_dev[64];
 
 // Once per device, with that device current: the arrays' device addresses
 // (in host code the array names are host-side stand-ins, not addresses).
-int noalloc_setup(int dev, NoAllocDevice** out)
+// Resolving a symbol may load the module, which a stream capture does not
+// allow, so the first call on a device is refused while `stream` is captured.
+int noalloc_setup(int dev, cudaStream_t stream, NoAllocDevice** out)
 {
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     NoAllocDevice& d = g_noalloc_dev[dev];
     if (!d.ready) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        NVFP4_CUDA_TRY(cudaStreamIsCapturing(stream, &cs));
+        if (cs != cudaStreamCaptureStatusNone) return NVFP4_ERR_CAPTURE;
         if (gemm_workspace_floats_per_warp() * kNoAllocMaxWarps > kNoAllocPartialFloats)
             return NVFP4_ERR_SCRATCH;
         void* p = nullptr;
@@ -80,7 +85,7 @@ extern "C" int nvfp4_gemm_decode_noalloc(const void* X, int M, const uint8_t* wq
     NVFP4_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return NVFP4_ERR_ARG;
     NoAllocDevice* d = nullptr;
-    st = noalloc_setup(dev, &d);
+    st = noalloc_setup(dev, (cudaStream_t)stream, &d);
     if (st != NVFP4_OK) return st;
     DeviceState ds;
     ds.device = dev;
@@ -91,7 +96,10 @@ extern "C" int nvfp4_gemm_decode_noalloc(const void* X, int M, const uint8_t* wq
     long long warps = 0;
     st = gemm_launch_warps(a, &ds, &warps);
     if (st != NVFP4_OK) return st;
-    if (warps > kNoAllocMaxWarps) return NVFP4_ERR_SCRATCH;
+    // A launch that would use more warps than the array holds runs with fewer
+    // (launch_gemm clamps the grid to ds.max_warps; the split-K partition stays
+    // correct for any warp count), so no shape is refused for its size.
+    if (warps > kNoAllocMaxWarps) warps = kNoAllocMaxWarps;
     // The array keeps the last call's contents: the arrival counters must start at zero.
     NVFP4_CUDA_TRY(cudaMemsetAsync(d->counters, 0, (size_t)warps * sizeof(unsigned), (cudaStream_t)stream));
     return launch_gemm(a, (cudaStream_t)stream, false, &ds);
