@@ -17,12 +17,14 @@
 // one mbarrier per stage, dequantises in registers and feeds bf16 m16n8k16
 // tensor-core MMAs with the lanes of X as the 8-wide N side.  A tile
 // (32 rows) that straddles warp ranges is finished by whichever of its
-// contributors arrives last: each writes its partial sums to the workspace,
-// bumps the tile's counter, and the last one adds the partials in warp order
-// (fixed, so results are bit-identical run to run) and runs the epilogue.
-// In the plain and fused kernels no thread ever waits on another warp or
-// CTA; the persistent round kernel at the end of the file is the one place
-// where the grid meets, at a bounded barrier between nodes.
+// contributors arrives last, in two levels (finish_tile): the contributors
+// inside one CTA count in at a shared-memory counter and the last of them adds
+// their partial sums in warp order; a tile that spans CTAs then has each CTA's
+// sum counted in at a global counter, and the last CTA adds them in CTA order.
+// Both orders are fixed, so results are bit-identical run to run.  In the
+// plain and fused kernels no thread ever waits on another warp or CTA; the
+// persistent round kernel at the end of the file is the one place where the
+// grid meets, at a bounded barrier between nodes.
 //
 // PDL: every kernel signals its dependents at entry, issues its weight
 // copies (which depend on nothing), and only then waits for the preceding
@@ -48,11 +50,6 @@ constexpr int kWarps = 16;                 // warps per CTA at M <= 8 (one CTA p
 constexpr int kMinBlocks = 1;              // CTAs per SM the register budget is sized for
 constexpr int kSlotFloats = 512;           // partial-sum slot: 2 matrices x 32 rows x 8 lanes
 
-// Partial-sum slot stride for NA accumulator sets per lane (32 lanes x 8
-// floats each): kSlotFloats up to two sets, twice that up to four (kernels
-// with four sets run half as many warps, so the workspace holds them).
-template <int NA>
-constexpr int kSlotStride = NA <= 2 ? kSlotFloats : 2 * kSlotFloats;
 
 struct KParams {
     const uint8_t* wq[2];
@@ -64,7 +61,31 @@ struct KParams {
     long long total_warps;
     float* partials;
     unsigned* counters;
+    long long rb_q;  // units / total_warps
+    unsigned rb_r;   // units % total_warps
+    float* legacy_partials;  // the fused kernel's one-level combine (plain floats, its own region)
 };
+
+// range_begin(units, total_warps, w) of the decode kernels without a 64-bit
+// division: q*w + (r*w)/TW, with r*w < 2^32 (total_warps < 2^16).
+__device__ __forceinline__ long long kp_begin(const KParams& p, long long w)
+{
+    return p.rb_q * w + (long long)((unsigned)p.rb_r * (unsigned)w / (unsigned)p.total_warps);
+}
+
+// range_owner(units, total_warps, x) for x < units: a double-precision
+// estimate of ((x+1)*TW - 1) / units (numerator < 2^53, so off by at most one)
+// corrected to the exact quotient.
+__device__ __forceinline__ long long kp_owner(const KParams& p, long long x)
+{
+    const long long n = (x + 1) * p.total_warps - 1;
+    long long w = (long long)((double)n / (double)p.units);
+    if ((w + 1) * p.units <= n)
+        ++w;
+    else if (w * p.units > n)
+        --w;
+    return w;
+}
 
 // 32 bytes of X into x when `pred`; x keeps its contents otherwise.
 __device__ __forceinline__ void ld_x32_keep(const void* p, bool pred, uint32_t (&x)[8])
@@ -150,9 +171,6 @@ __device__ __forceinline__ void epilogue(const OutArgs& o, long long tile, const
         }
 }
 
-// One lane's share of a unit: X fragments are in xw; sq and ss point at the
-// lane's code bytes and scale word in shared memory.  Adds the unit's products into acc.
-
 // Load one contributor's partial sums (this lane's NW*8 floats).
 template <int NW>
 __device__ __forceinline__ void load_partial(const float* src, float4 (&v)[NW * 2])
@@ -161,7 +179,92 @@ __device__ __forceinline__ void load_partial(const float* src, float4 (&v)[NW * 
     for (int k = 0; k < NW * 2; ++k) v[k] = ld_cg_f4(src + 4 * k);
 }
 
-// End of a tile for this warp, after it stored its sums in its partial slot.
+// The persistent round kernel's combine, through the workspace only: end of a
+// tile for this warp, after it stored its sums in its partial slot.  A tile
+// the warp covered alone goes straight to the epilogue.  Otherwise the warp
+// counts itself in, and the last contributor adds the partials in the order
+// the decode kernel's two-level combine uses -- each CTA's contributors in
+// warp order, then those CTA sums in CTA order -- so a GEMM node of the
+// persistent round equals a direct call bit for bit.  Out of line, so the
+// streaming loop does not carry its registers.
+template <int M>
+__device__ __noinline__ void tile_done_round(const OutArgs o, long long tile, int lane)
+{
+    const long long U = o.units, TW = o.total_warps, KC = o.k_chunks;
+    const long long ts = tile * KC, te = ts + KC;
+    const long long glo = range_owner(U, TW, ts), ghi = range_owner(U, TW, te - 1);
+    if (glo != ghi) {
+        // The lanes' partial stores are ordered before lane 0's release by the
+        // warp barrier; the acquire side orders the last contributor's reads
+        // of the other partials after theirs.
+        __syncwarp();
+        unsigned last = 0;
+        if (lane == 0) {
+            unsigned old;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(o.counters + glo) : "memory");
+            last = (old == (unsigned)(ghi - glo)) ? 1u : 0u;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) return;
+    }
+    const int glo_slot = (range_begin(U, TW, glo) >= ts) ? 0 : 1;
+    float total[1][2][4], local[1][2][4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) total[0][r][i] = local[0][r][i] = 0.f;
+    long long cta = glo / kWarps;
+    constexpr int kBatch = 4;  // contributors whose loads are in flight together
+    for (long long w0 = glo; w0 <= ghi; w0 += kBatch) {
+        float4 v[kBatch][2];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const long long w = w0 + b;
+            if (w <= ghi) {
+                const int ws = (w == glo) ? glo_slot : 0;
+                load_partial<1>(o.partials + ((size_t)w * 2 + ws) * kSlotFloats + lane * 8, v[b]);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const long long w = w0 + b;
+            if (w <= ghi) {
+                if (w / kWarps != cta) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            total[0][r][i] += local[0][r][i];
+                            local[0][r][i] = 0.f;
+                        }
+                    cta = w / kWarps;
+                }
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    local[0][r][0] += v[b][r].x;
+                    local[0][r][1] += v[b][r].y;
+                    local[0][r][2] += v[b][r].z;
+                    local[0][r][3] += v[b][r].w;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) total[0][r][i] += local[0][r][i];
+    epilogue<M, 1>(o, tile, total, lane >> 2, lane & 3);
+    if (glo != ghi && lane == 0) atomicExch(&o.counters[glo], 0u);
+}
+
+// Slot stride of the one-level combine for NA accumulator sets per lane.
+template <int NA>
+constexpr int kLegacyStride = NA <= 2 ? kSlotFloats : 2 * kSlotFloats;
+
+// The fused gate/up kernel's combine, one level through the workspace (its
+// streaming loop sits at the register limit, with no room for the two-level
+// combine's bookkeeping): end of a tile for this warp, after it stored its
+// sums in its partial slot of the legacy region.
 // A tile the warp covered alone goes straight to the epilogue.  Otherwise the
 // warp counts itself in, and the last contributor adds every partial in warp
 // order (glo..ghi, a fixed order, so the result does not depend on who arrives
@@ -174,7 +277,7 @@ __device__ __forceinline__ void load_partial(const float* src, float4 (&v)[NW * 
 // into registers a few at a time, the first few while the copies are in
 // flight.  Out of line, so the streaming loop does not carry its registers.
 template <int M, int NW>
-__device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane, uint32_t gather_smem,
+__device__ __noinline__ void tile_done_global(const OutArgs o, long long tile, int lane, uint32_t gather_smem,
                                        uint32_t gather_bytes, uint32_t gather_bar)
 {
     constexpr int NA = kAccSets<M, NW>;  // accumulator sets per lane in a partial
@@ -230,7 +333,7 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
             const long long w = glo + c;
             const int ws = (w == glo) ? glo_slot : 0;
             const uint64_t pol = evict_first_policy();
-            bulk_load(gather_smem + c * kPartBytes, o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA>, kPartBytes,
+            bulk_load(gather_smem + c * kPartBytes, o.partials + ((size_t)w * 2 + ws) * kLegacyStride<NA>, kPartBytes,
                       gather_bar, pol);
         }
     }
@@ -242,7 +345,7 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
         const long long w = w0 + b;
         if (w <= ghi) {
             const int ws = (w == glo) ? glo_slot : 0;
-            load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), v[b]);
+            load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kLegacyStride<NA> + lane * (NA * 8), v[b]);
         }
     }
     if (nb > 0) {
@@ -272,7 +375,7 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
                     } else {
                         const long long w = glo + c + e;
                         const int ws = (w == glo) ? glo_slot : 0;
-                        load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), x[e]);
+                        load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kLegacyStride<NA> + lane * (NA * 8), x[e]);
                     }
                 }
             }
@@ -310,12 +413,341 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
             const long long w = w0 + b;
             if (w <= ghi) {
                 const int ws = (w == glo) ? glo_slot : 0;
-                load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kSlotStride<NA> + lane * (NA * 8), v[b]);
+                load_partial<NA>(o.partials + ((size_t)w * 2 + ws) * kLegacyStride<NA> + lane * (NA * 8), v[b]);
             }
         }
     }
     epilogue<M, NW>(o, tile, sum, lane >> 2, lane & 3);
     if (glo != ghi && lane == 0) atomicExch(&o.counters[glo], 0u);
+}
+
+
+// ------------------------------------------------------------------ the combine of the decode kernels
+//
+// Warp gw owns units [kp_begin(gw), kp_begin(gw + 1)); CTA c owns the union of
+// its warps' ranges, [uc, uc1).  A tile with several contributors is summed by
+// a designated finisher, first inside each CTA, then across CTAs:
+//   - inside a CTA, the finisher is the last contributor whose range ends in
+//     the tile.  A contributor whose range ends in the tile leaves its partial
+//     sums in its own ring (idle from then on) and raises its shared-memory
+//     flag; the one contributor that may leave the tile in mid-range (the
+//     tile's last in the CTA) writes them to a slot of the CTA's shared-memory
+//     pool (slot = the tile's index among the CTA's tiles) and raises its
+//     other flag, or, when the CTA spans more tiles than the pool has slots,
+//     to its workspace slot 0;
+//   - across CTAs, the finisher is the one of the CTA that holds the tile's
+//     first unit; every other CTA's sum goes to one of that CTA's two CTA
+//     slots.
+// Workspace slots hold LL words: 64 bits, a float's bits below a ready flag, so
+// a 64-bit store publishes data and flag together and the reader polls the
+// data itself -- no fence, no atomic, no release on the writer's side, which at
+// GPU scope would cost a round trip to L2 under load.  The reader clears each
+// slot it consumed, so every slot is zero when the next launch starts.  A
+// finisher waits only for warps of higher index, and those never wait for it,
+// so the waits form no cycle; all CTAs of the grid are resident (one per SM,
+// at most as many as SMs), and every wait is bounded.  Sums run in warp order
+// inside a CTA and in CTA order across, so results are bit-identical run to run.
+
+// Workspace slot s of warp w: [lane][NA * 8] LL words.
+template <int NA>
+__device__ __forceinline__ uint64_t* ll_slot(const KParams& p, long long w, int s)
+{
+    return reinterpret_cast<uint64_t*>(p.partials) + ((size_t)w * 2 + s) * (NA * 256);
+}
+
+// Slot of CTA c's sum of `tile`: slot 1 of the CTA's first warp for the last
+// tile of its range, of its second warp for the first (slot 1 of a warp is
+// used for nothing else).
+template <int W, int NA>
+__device__ __forceinline__ uint64_t* cta_slot(const KParams& p, long long c, long long tile)
+{
+    const long long w1 = (c + 1) * W < p.total_warps ? (c + 1) * W : p.total_warps;
+    const long long last_tile = (kp_begin(p, w1) - 1) / p.k_chunks;
+    return ll_slot<NA>(p, c * W + (tile == last_tile ? 0 : 1), 1);
+}
+
+constexpr unsigned long long kLLReady = 1ull << 32;
+
+template <int NA>
+__device__ __forceinline__ void ll_write(uint64_t* slot, int lane, const float (&acc)[NA][2][4])
+{
+    uint64_t* d = slot + lane * (NA * 8);
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; i += 2)
+                asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(d + (a * 2 + r) * 4 + i),
+                             "l"(kLLReady | __float_as_uint(acc[a][r][i])),
+                             "l"(kLLReady | __float_as_uint(acc[a][r][i + 1]))
+                             : "memory");
+}
+
+// Poll slot (bounded) until every word carries the ready flag, add its
+// floats into sum, and clear the slot for the next launch.  Returns false if
+// the wait gave up.
+template <int NA>
+__device__ __forceinline__ bool ll_read_add(uint64_t* slot, int lane, float (&sum)[NA][2][4])
+{
+    uint64_t* d = slot + lane * (NA * 8);
+    unsigned long long v[NA * 8];
+    bool ok = false;
+    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+        bool ready = true;
+#pragma unroll
+        for (int k = 0; k < NA * 8; k += 2) {
+            asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(v[k]), "=l"(v[k + 1]) : "l"(d + k) : "memory");
+            ready = ready && (v[k] >> 32) == 1u && (v[k + 1] >> 32) == 1u;
+        }
+        if (__all_sync(0xffffffffu, ready)) {
+            ok = true;
+            break;
+        }
+        __nanosleep(64);
+    }
+#pragma unroll
+    for (int k = 0; k < NA * 8; ++k) sum[k >> 3][(k >> 2) & 1][k & 3] += __uint_as_float((unsigned)v[k]);
+#pragma unroll
+    for (int k = 0; k < NA * 8; k += 2)
+        asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(d + k), "l"(0ull), "l"(0ull) : "memory");
+    return ok;
+}
+
+template <int NA>
+__device__ __forceinline__ void store_ring_partial(uint32_t ring, int lane, const float (&acc)[NA][2][4])
+{
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(ring + (uint32_t)(((a * 2 + r) * 32 + lane) * 16)),
+                         "f"(acc[a][r][0]), "f"(acc[a][r][1]), "f"(acc[a][r][2]), "f"(acc[a][r][3])
+                         : "memory");
+}
+
+template <int NA>
+__device__ __forceinline__ void add_ring_partial(uint32_t ring, int lane, float (&sum)[NA][2][4])
+{
+#pragma unroll
+    for (int k = 0; k < NA * 2; ++k) {
+        float4 x;
+        asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                     : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                     : "r"(ring + (uint32_t)((k * 32 + lane) * 16))
+                     : "memory");
+        sum[k >> 1][k & 1][0] += x.x;
+        sum[k >> 1][k & 1][1] += x.y;
+        sum[k >> 1][k & 1][2] += x.z;
+        sum[k >> 1][k & 1][3] += x.w;
+    }
+}
+
+template <int NA>
+__device__ __forceinline__ void add_into(float (&sum)[NA][2][4], const float4 (&x)[NA * 2])
+{
+#pragma unroll
+    for (int k = 0; k < NA * 2; ++k) {
+        sum[k >> 1][k & 1][0] += x[k].x;
+        sum[k >> 1][k & 1][1] += x[k].y;
+        sum[k >> 1][k & 1][2] += x[k].z;
+        sum[k >> 1][k & 1][3] += x[k].w;
+    }
+}
+
+template <int M, int NW>
+__device__ __forceinline__ void epilogue_p(const KParams& p, long long tile, const float (&acc)[kAccSets<M, NW>][2][4],
+                                           int g, int t)
+{
+    OutArgs o;
+    o.out = p.out;
+    o.N = p.N;
+    o.gs0 = p.gs[0];
+    o.gs1 = p.gs[1];
+    epilogue<M, NW>(o, tile, acc, g, t);
+}
+
+// Dynamic shared memory of a decode kernel: the warps' rings, their stage
+// barriers, the pool of mid-range partial sums, the flags (ring partial ready
+// [0, W), pool partial ready [W, 2W)) and the warps' unit boundaries.
+template <int NA>
+struct AccPack {
+    float v[NA][2][4];
+};
+
+constexpr int kSmemPerBlock = 227 * 1024;
+
+template <int M, int NW, int STAGES, int UPS, int W>
+struct SmemLayout {
+    static constexpr int kStage = NW * UPS * kUnitBytes;
+    static constexpr int kRings = W * STAGES * kStage;
+    static constexpr int kBars = kRings;                       // W * STAGES mbarriers
+    static constexpr int kPool = kBars + W * STAGES * 8;
+    static constexpr int kSlot = kAccSets<M, NW> * 1024;        // one partial: NA x 32 lanes x 8 floats
+    static constexpr int kTail = 2 * W * 4 + (W + 1) * 8 + 64;  // flags, boundaries, alignment slack
+    static constexpr int kFit = (kSmemPerBlock - kPool - kTail) / kSlot;
+    static constexpr int kPoolSlots = NW == 2 ? 0 : kFit < 0 ? 0 : kFit > 8 ? 8 : kFit;  // at most 8
+    static constexpr int kGather = kPool + kPoolSlots * kSlot;   // NW == 2: one gather mbarrier per warp
+    static constexpr int kFlags = kGather + (NW == 2 ? W * 8 : 0);
+    static constexpr int kWb = kFlags + 2 * W * 4;              // 8-byte aligned: kFlags is a multiple of 8
+    static constexpr int kBytes = kWb + (W + 1) * 8;
+    static_assert(kBytes <= kSmemPerBlock, "shared memory over budget");
+};
+
+// The warp of this CTA whose range holds unit x (uc <= x < uc1): wb[w] is the
+// first unit of local warp w, wb[W] = uc1 (a binary search over W + 1 entries).
+template <int W>
+__device__ __forceinline__ int local_owner(const long long* wb, long long x)
+{
+    int lo = 0, hi = W;
+#pragma unroll
+    for (int s = 0; s < 5; ++s)
+        if (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (wb[mid] <= x)
+                lo = mid;
+            else
+                hi = mid;
+        }
+    return lo;
+}
+
+// The designated finisher of `tile` in this CTA (its own partial is already
+// in its ring): add the CTA's partials in warp order, then either run the
+// epilogue (the tile lies in this CTA), publish the CTA's sum (another CTA
+// finishes the tile), or add the other CTAs' sums in CTA order and run the
+// epilogue.
+template <int M, int NW, int STAGES, int UPS, int W>
+__device__ __noinline__ void finish_tile(const KParams& p, long long tile, int self, int lane)
+{
+    using L = SmemLayout<M, NW, STAGES, UPS, W>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int NA = kAccSets<M, NW>;
+    constexpr int POOL = L::kPoolSlots;
+    const uint32_t base = smem_addr(smem);
+    const uint32_t flags_s = base + L::kFlags, pool_s = base + L::kPool;
+    const long long* wb = reinterpret_cast<const long long*>(smem + L::kWb);
+    const long long cta = blockIdx.x, uc = wb[0], uc1 = wb[W];
+    const long long KC = p.k_chunks;
+    const long long ts = tile * KC, te = ts + KC;
+    const long long a = ts > uc ? ts : uc, b = te < uc1 ? te : uc1;
+    const int wlo = local_owner<W>(wb, a), whi = local_owner<W>(wb, b - 1);
+    const bool whi_crosses = wb[whi + 1] > b;
+    const long long ps = tile - uc / KC;  // the crossing contributor's pool slot
+    const bool cross_ll = whi_crosses && ps >= POOL;
+    // 1. every flag at once: lane i watches contributor wlo + i
+    bool ok;
+    {
+        const int v = wlo + lane;
+        bool done = true;
+        uint32_t f = 0;
+        if (v <= whi && v != self && !(v == whi && cross_ll)) {
+            done = false;
+            f = flags_s + 4u * (uint32_t)((v == whi && whi_crosses) ? W + v : v);
+        }
+        for (uint32_t it = 0; it < kWaitLimit; ++it) {
+            if (!done) {
+                uint32_t up;
+                asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(up) : "r"(f) : "memory");
+                done = up != 0;
+            }
+            if (__all_sync(0xffffffffu, done)) break;
+            __nanosleep(32);
+        }
+        ok = __all_sync(0xffffffffu, done);
+        // the lanes' acquires order every lane's reads below after the contributors' writes
+        __syncwarp();
+    }
+    // 2. the partials in warp order, 4 / NA contributors' loads in flight at a time
+    float sum[NA][2][4];
+#pragma unroll
+    for (int x = 0; x < NA; ++x)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sum[x][r][i] = 0.f;
+    constexpr int kB = NA >= 4 ? 1 : 4 / NA;
+    const int last_smem = cross_ll ? whi - 1 : whi;
+    for (int v0 = wlo; v0 <= last_smem; v0 += kB) {
+        float4 x[kB][NA * 2];
+#pragma unroll
+        for (int bb = 0; bb < kB; ++bb) {
+            const int v = v0 + bb;
+            if (v <= last_smem) {
+                const uint32_t src = (v == whi && whi_crosses) ? pool_s + (uint32_t)ps * L::kSlot
+                                                               : base + (uint32_t)v * (STAGES * L::kStage);
+#pragma unroll
+                for (int k = 0; k < NA * 2; ++k)
+                    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                 : "=f"(x[bb][k].x), "=f"(x[bb][k].y), "=f"(x[bb][k].z), "=f"(x[bb][k].w)
+                                 : "r"(src + (uint32_t)((k * 32 + lane) * 16))
+                                 : "memory");
+            }
+        }
+#pragma unroll
+        for (int bb = 0; bb < kB; ++bb)
+            if (v0 + bb <= last_smem) add_into<NA>(sum, x[bb]);
+    }
+    if (cross_ll) ok = ll_read_add<NA>(ll_slot<NA>(p, cta * W + whi, 0), lane, sum) && ok;
+    const long long clo = kp_owner(p, ts) / W, chi = kp_owner(p, te - 1) / W;
+    if (clo != chi) {
+        if (cta != clo) {
+            ll_write<NA>(cta_slot<W, NA>(p, cta, tile), lane, sum);
+            if (!ok && lane == 0) atomicOr(&g_device_status, 4u);
+            return;
+        }
+        for (long long c = clo + 1; c <= chi; ++c) ok = ll_read_add<NA>(cta_slot<W, NA>(p, c, tile), lane, sum) && ok;
+    }
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) atomicOr(&g_device_status, 4u);
+    epilogue_p<M, NW>(p, tile, sum, lane >> 2, lane & 3);
+}
+
+// This warp is done with its part of `tile` (at the tile's last chunk or the
+// end of its range), its sums in acc.  Out of line, so the streaming loop
+// carries none of its registers.
+template <int M, int NW, int STAGES, int UPS, int W>
+__device__ __noinline__ void flush_tile(const KParams& p, long long tile, const AccPack<kAccSets<M, NW>> acc, int lane,
+                                        int warp)
+{
+    using L = SmemLayout<M, NW, STAGES, UPS, W>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int NA = kAccSets<M, NW>;
+    const long long* wb = reinterpret_cast<const long long*>(smem + L::kWb);
+    const uint32_t base = smem_addr(smem);
+    const long long cta = blockIdx.x, KC = p.k_chunks;
+    const long long uc = wb[0], uc1 = wb[W], w0 = wb[warp], w1 = wb[warp + 1];
+    const long long ts = tile * KC, te = ts + KC;
+    const long long a = ts > uc ? ts : uc, b = te < uc1 ? te : uc1;  // the tile's units in this CTA
+    const bool alone = a >= w0 && b <= w1;  // this warp is the tile's only contributor in the CTA
+    if (alone && ts >= uc && te <= uc1) {
+        epilogue_p<M, NW>(p, tile, acc.v, lane >> 2, lane & 3);  // and the only one at all
+    } else if (w1 > b) {
+        // Leaves the tile in mid-range: publish the partial and go on (no wait, no
+        // fence): to the CTA's pool when it has the slot, else to the workspace.
+        const long long ps = tile - uc / KC;
+        if (!alone && ps < L::kPoolSlots) {
+            store_ring_partial<NA>(base + L::kPool + (uint32_t)ps * L::kSlot, lane, acc.v);
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("st.release.cta.shared::cta.u32 [%0], 1;" ::"r"(base + L::kFlags + 4u * (W + warp))
+                             : "memory");
+        } else {
+            ll_write<NA>(alone ? cta_slot<W, NA>(p, cta, tile) : ll_slot<NA>(p, cta * W + warp, 0), lane, acc.v);
+        }
+    } else {
+        // Its range ends in the tile: every stage is consumed and the ring is idle.
+        store_ring_partial<NA>(base + (uint32_t)warp * (STAGES * L::kStage), lane, acc.v);
+        // the designated finisher: the last contributor in the CTA whose range ends here
+        const int whi = local_owner<W>(wb, b - 1);
+        const int fin = wb[whi + 1] > b ? whi - 1 : whi;
+        if (warp == fin) {
+            finish_tile<M, NW, STAGES, UPS, W>(p, tile, warp, lane);
+        } else {
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("st.release.cta.shared::cta.u32 [%0], 1;" ::"r"(base + L::kFlags + 4u * warp) : "memory");
+        }
+    }
 }
 
 // STAGES shared-memory stages per warp, each holding UPS consecutive units of
@@ -324,44 +756,55 @@ __device__ __noinline__ void tile_done(const OutArgs o, long long tile, int lane
 // of the MMA's 8-wide side, and every dequantised word feeds each block.
 template <int M, int NW, int STAGES, int UPS, int W>
 __global__ void __launch_bounds__(W * 32, kMinBlocks)
-decode_gemm_kernel(const KParams p)
+decode_gemm_kernel(const __grid_constant__ KParams p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
+    using L = SmemLayout<M, NW, STAGES, UPS, W>;
     constexpr int kMatStage = UPS * kUnitBytes;
     constexpr int kStage = NW * kMatStage;
     constexpr int NB = (M + 7) / 8;        // blocks of 8 decode lanes
     constexpr int NA = kAccSets<M, NW>;    // accumulator sets
+    unsigned* s_flag = reinterpret_cast<unsigned*>(smem + L::kFlags);
+    long long* s_wb = reinterpret_cast<long long*>(smem + L::kWb);  // warp w owns units [s_wb[w], s_wb[w + 1])
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const long long gw = (long long)blockIdx.x * W + warp;
+    const long long cta = blockIdx.x;
+    const long long gw = cta * W + warp;
 
     // Dependents may begin launching; they wait for this grid before using its results.
     asm volatile("griddepcontrol.launch_dependents;");
 
-    const long long U = p.units, TW = p.total_warps, KC = p.k_chunks;
+    if (threadIdx.x < 2 * W) s_flag[threadIdx.x] = 0u;
+    if (threadIdx.x <= W) {
+        const long long w = cta * W + threadIdx.x;
+        s_wb[threadIdx.x] = kp_begin(p, w < p.total_warps ? w : p.total_warps);
+    }
+    __syncthreads();
+    const long long TW = p.total_warps, KC = p.k_chunks;
     if (gw >= TW) return;
-    const long long u0 = range_begin(U, TW, gw), u1 = range_begin(U, TW, gw + 1);
-    const int n_units = (int)(u1 - u0);
+    // this warp's units [s_wb[warp], s_wb[warp + 1]), the CTA's [s_wb[0], s_wb[W]): read from
+    // shared memory where needed, so the streaming loop keeps none of them in registers
+    const long long u0 = s_wb[warp];
+    const int n_units = (int)(s_wb[warp + 1] - u0);
     const int n_stages = (n_units + UPS - 1) / UPS;
 
     uint8_t* ring = smem + warp * (STAGES * kStage);
     const uint32_t ring_s = smem_addr(ring);
     const uint32_t bar_s = smem_addr(smem + W * STAGES * kStage) + warp * STAGES * 8;
-    // one more mbarrier per warp, for gathering partial sums into the idle ring
-    const uint32_t gather_bar = smem_addr(smem + W * STAGES * (kStage + 8)) + warp * 8;
 
+    const uint32_t gather_bar = smem_addr(smem + L::kGather) + warp * 8;  // NW == 2 only
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) mbar_init(bar_s + 8 * s);
-        mbar_init(gather_bar);
+        if constexpr (NW == 2) mbar_init(gather_bar);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncwarp();
 
-    const uint64_t pol = evict_first_policy();
     auto issue = [&](int j, int slot) {
+        const uint64_t pol = evict_first_policy();  // made here: one register pair less across the loop
         const long long ub = u0 + (long long)j * UPS;
         const int rem = n_units - j * UPS;
         const int cnt = rem < UPS ? rem : UPS;
@@ -392,7 +835,7 @@ decode_gemm_kernel(const KParams p)
             for (int i = 0; i < 4; ++i) acc[a][r][i] = 0.f;
 
     long long tile = u0 / KC;
-    const long long first_tile = tile;
+    const long long first_tile = tile;  // NW == 2: the partial slot of a tile left in mid-range
     int chunk = (int)(u0 - tile * KC);
     const int kc_last = (int)KC - 1;
     const int K32 = (int)p.K;
@@ -467,28 +910,39 @@ decode_gemm_kernel(const KParams p)
                 ++i;
                 const bool tile_end = chunk == kc_last;
                 if (tile_end || i == n_units) {
-                    // Partial slot: 0 for the tile this warp's range starts in, 1 for a later one.
-                    const int slot_id = (tile == first_tile) ? 0 : 1;
-                    float* dst = p.partials + ((size_t)gw * 2 + slot_id) * kSlotStride<NA> + lane * (NA * 8);
+                    if constexpr (NW == 2) {
+                        // Partial slot: 0 for the tile this warp's range starts in, 1 for a later one.
+                        const int slot_id = (tile == first_tile) ? 0 : 1;
+                        float* dst = p.legacy_partials + ((size_t)gw * 2 + slot_id) * kLegacyStride<NA> + lane * (NA * 8);
 #pragma unroll
-                    for (int a = 0; a < NA; ++a)
+                        for (int a = 0; a < NA; ++a)
 #pragma unroll
-                        for (int r = 0; r < 2; ++r)
-                            reinterpret_cast<float4*>(dst)[a * 2 + r] =
-                                make_float4(acc[a][r][0], acc[a][r][1], acc[a][r][2], acc[a][r][3]);
-                    OutArgs o;
-                    o.out = p.out;
-                    o.partials = p.partials;
-                    o.counters = p.counters;
-                    o.N = p.N;
-                    o.units = p.units;
-                    o.total_warps = p.total_warps;
-                    o.k_chunks = p.k_chunks;
-                    o.gs0 = p.gs[0];
-                    o.gs1 = p.gs[1];
-                    // At the end of the range every stage has been consumed and no copy is
-                    // in flight, so the ring can take the partial sums of a combine.
-                    tile_done<M, NW>(o, tile, lane, i == n_units ? ring_s : 0u, STAGES * kStage, gather_bar);
+                            for (int r = 0; r < 2; ++r)
+                                reinterpret_cast<float4*>(dst)[a * 2 + r] =
+                                    make_float4(acc[a][r][0], acc[a][r][1], acc[a][r][2], acc[a][r][3]);
+                        OutArgs o;
+                        o.out = p.out;
+                        o.partials = p.legacy_partials;
+                        o.counters = p.counters;
+                        o.N = p.N;
+                        o.units = p.units;
+                        o.total_warps = p.total_warps;
+                        o.k_chunks = p.k_chunks;
+                        o.gs0 = p.gs[0];
+                        o.gs1 = p.gs[1];
+                        // At the end of the range every stage has been consumed and no copy is
+                        // in flight, so the ring can take the partial sums of a combine.
+                        tile_done_global<M, NW>(o, tile, lane, i == n_units ? ring_s : 0u, STAGES * kStage, gather_bar);
+                    } else {
+                        AccPack<NA> pk;
+#pragma unroll
+                        for (int x = 0; x < NA; ++x)
+#pragma unroll
+                            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) pk.v[x][r][k] = acc[x][r][k];
+                        flush_tile<M, NW, STAGES, UPS, W>(p, tile, pk, lane, warp);
+                    }
 #pragma unroll
                     for (int a = 0; a < NA; ++a)
 #pragma unroll
@@ -706,7 +1160,7 @@ __device__ __forceinline__ bool round_gemm(const RoundParams& rp, const RoundNod
                         o.k_chunks = vn->k_chunks;
                         o.gs0 = vn->gs[0];
                         o.gs1 = vn->gs[1];
-                        tile_done<M, 1>(o, tile, lane, 0u, 0u, 0u);
+                        tile_done_round<M>(o, tile, lane);
 #pragma unroll
                         for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -874,14 +1328,16 @@ struct KernelOf {
     static constexpr int stages = wide ? kStagesWide : NW == 2 ? kStagesFused : SHORT ? kStagesPlainShort : kStagesPlain;
     static constexpr int ups = wide ? wide_units_per_stage(nb)
                                : NW == 2 ? kUnitsPerStageFused : SHORT ? kUnitsPerStagePlainShort : kUnitsPerStagePlain;
+    static constexpr int acc_sets = kAccSets<M, NW>;
     static void* fn() { return (void*)decode_gemm_kernel<M, NW, stages, ups, warps>; }
-    static size_t smem() { return (size_t)warps * stages * (NW * ups * kUnitBytes + 8) + warps * 8; }
+    static size_t smem() { return SmemLayout<M, NW, stages, ups, warps>::kBytes; }
 };
 
 struct KernelInfo {
     void* fn = nullptr;
     size_t smem = 0;
     int warps = 0;
+    int acc_sets = 0;       // accumulator sets per lane: a workspace slot holds acc_sets * 512 floats
     int blocks_per_sm = 0;  // filled on first use
 };
 
@@ -897,6 +1353,7 @@ KernelInfo kernel_info_for(int M, bool short_stages)
         k.fn = KernelOf<m, 1, true>::fn();                 \
         k.smem = KernelOf<m, 1, true>::smem();             \
         k.warps = KernelOf<m, 1, true>::warps;             \
+        k.acc_sets = KernelOf<m, 1, true>::acc_sets;       \
         return k;
                 NVFP4_SHORT(5) NVFP4_SHORT(6) NVFP4_SHORT(7) NVFP4_SHORT(8)
 #undef NVFP4_SHORT
@@ -910,6 +1367,7 @@ KernelInfo kernel_info_for(int M, bool short_stages)
         k.fn = KernelOf<m, NW>::fn();        \
         k.smem = KernelOf<m, NW>::smem();    \
         k.warps = KernelOf<m, NW>::warps;    \
+        k.acc_sets = KernelOf<m, NW>::acc_sets; \
         break;
         NVFP4_CASE(1) NVFP4_CASE(2) NVFP4_CASE(3) NVFP4_CASE(4)
         NVFP4_CASE(5) NVFP4_CASE(6) NVFP4_CASE(7) NVFP4_CASE(8)
@@ -955,13 +1413,17 @@ int device_state(cudaStream_t stream, DeviceState** out)
     const int max_warps = sms * (max_threads / 32);
     float* partials = nullptr;
     unsigned* counters = nullptr;
-    NVFP4_CUDA_TRY(cudaMalloc(&partials, (size_t)max_warps * 2 * kSlotFloats * sizeof(float)));
+    // two regions: the decode kernels' slots (which must start zeroed: their
+    // ready flags), then the persistent round kernel's
+    const size_t region = (size_t)max_warps * 2 * kSlotFloats;
+    NVFP4_CUDA_TRY(cudaMalloc(&partials, 2 * region * sizeof(float)));
     cudaError_t e = cudaMalloc(&counters, (size_t)max_warps * sizeof(unsigned));
     if (e != cudaSuccess) {
         cudaFree(partials);
         return fail_cuda(e);
     }
     e = cudaMemset(counters, 0, (size_t)max_warps * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemset(partials, 0, region * sizeof(float));
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         cudaFree(partials);
@@ -971,6 +1433,7 @@ int device_state(cudaStream_t stream, DeviceState** out)
     s.sm_count = sms;
     s.max_warps = max_warps;
     s.partials = partials;
+    s.round_partials = partials + region;
     s.counters = counters;
     s.device = dev;
     *out = &s;
@@ -1041,7 +1504,11 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
     long long ctas = (long long)ds->sm_count * k->blocks_per_sm;
     const long long need = (geo.units + W - 1) / W;
     if (need < ctas) ctas = need;
-    if (ctas * W > ds->max_warps) ctas = ds->max_warps / W;
+    // The workspace holds max_warps warps of two 512-float slots; a warp of this
+    // kernel takes acc_sets times that.
+    const long long per_cta = (long long)W * k->acc_sets;
+    if (ctas * per_cta > ds->max_warps) ctas = ds->max_warps / per_cta;
+    if (ctas < 1) return NVFP4_ERR_SCRATCH;
     // Never more warps than units: every warp below total_warps gets a
     // non-empty range (the split-K combine relies on it).
     const long long total_warps = ctas * W < geo.units ? ctas * W : geo.units;
@@ -1062,6 +1529,10 @@ int launch_gemm(const GemmArgs& a, cudaStream_t stream, bool pdl, DeviceState* d
     p.total_warps = total_warps;
     p.partials = ds->partials;
     p.counters = ds->counters;
+    if (total_warps >= (1 << 16)) return NVFP4_ERR_SHAPE;  // kp_begin keeps r * w below 2^32
+    p.legacy_partials = ds->round_partials;
+    p.rb_q = geo.units / total_warps;
+    p.rb_r = (unsigned)(geo.units % total_warps);
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ctas);
@@ -1171,7 +1642,7 @@ int round_persistent_build(const GemmArgs* nodes, int n, DeviceState* ds, float*
         }
     }
     rp->n_nodes = k;
-    rp->partials = ds->partials;
+    rp->partials = ds->round_partials;
     rp->counters = ds->counters;
     *count = k;
     return NVFP4_OK;
@@ -1235,9 +1706,14 @@ int read_and_clear_device_status(int* status)
         int dev = 0;
         NVFP4_CUDA_TRY(cudaGetDevice(&dev));
         std::lock_guard<std::mutex> lock(g_mu);
-        if (dev >= 0 && dev < 64 && g_states[dev].device == dev)
+        if (dev >= 0 && dev < 64 && g_states[dev].device == dev) {
+            // a wait that gave up may have left counters raised and slots unconsumed
             NVFP4_CUDA_TRY(cudaMemset(g_states[dev].counters, 0,
                                       (size_t)g_states[dev].max_warps * sizeof(unsigned)));
+            NVFP4_CUDA_TRY(cudaMemset(g_states[dev].partials, 0,
+                                      (size_t)g_states[dev].max_warps * 2 * kSlotFloats * sizeof(float)));
+        }
+        NVFP4_CUDA_TRY(noalloc_clear_scratch());
         NVFP4_CUDA_TRY(cudaDeviceSynchronize());
     }
     *status = (int)v;

@@ -34,7 +34,8 @@ struct DeviceState {
     int device = -1;
     int sm_count = 0;
     int max_warps = 0;        // capacity of the workspace, in warps
-    float* partials = nullptr;
+    float* partials = nullptr;        // the decode kernels' workspace slots (zeroed between launches)
+    float* round_partials = nullptr;  // the persistent round kernel's
     unsigned* counters = nullptr;
 };
 int device_state(cudaStream_t stream, DeviceState** out);
@@ -72,8 +73,11 @@ int round_persistent_build(const GemmArgs* nodes, int n, DeviceState* ds, float*
 int round_persistent_prepare(DeviceState* ds, int M, int* grid);
 int round_persistent_launch(void* params_host, unsigned* d_arrive, int M, int grid, cudaStream_t stream);
 
-// Device-side status word (nonzero after a bounded wait gave up).
+// Device-side status word (nonzero after a bounded wait gave up).  When it is
+// nonzero the workspaces are cleared, the no-allocation entry point's included
+// (noalloc_clear_scratch, a cudaError_t).
 int read_and_clear_device_status(int* status);
+cudaError_t noalloc_clear_scratch();
 
 // The decode GEMM at verify widths (M = kVerifyMinM..kVerifyMaxM) on the
 // tensor-memory path: geometry of a call, its launch, and its status word.

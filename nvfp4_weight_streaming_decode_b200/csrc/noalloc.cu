@@ -61,6 +61,25 @@ int noalloc_setup(int dev, cudaStream_t stream, NoAllocDevice** out)
 }
 
 }  // namespace
+
+// After a bounded wait gave up, slots may be left unconsumed: zero the
+// array on every device whose address was resolved (current device restored).
+cudaError_t noalloc_clear_scratch()
+{
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    int cur = 0;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return e;
+    for (int dev = 0; dev < 64; ++dev) {
+        if (!g_noalloc_dev[dev].ready) continue;
+        e = cudaSetDevice(dev);
+        if (e == cudaSuccess) e = cudaMemset(g_noalloc_dev[dev].partials, 0, kNoAllocPartialFloats * sizeof(float));
+        if (e != cudaSuccess) break;
+    }
+    const cudaError_t e2 = cudaSetDevice(cur);
+    return e != cudaSuccess ? e : e2;
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;

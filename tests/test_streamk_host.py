@@ -67,3 +67,98 @@ def test_lane_block_x_rows_stay_inside_x(M):
             assert 0 <= r < M, (M, g, b, r)
             if 8 * b + g < M:
                 assert r == 8 * b + g
+
+
+def _combine_plan(n_tiles, k_chunks, TW, W, POOL):
+    """Replay, for every warp, what the decode kernel does when it is done
+    with its part of a tile (the flush site and finish_tile), in the kernel's
+    integer formulas.  Returns the writes (location -> (tile, writer)), the
+    epilogues run per tile, and the reads and waits of every finisher."""
+    U = n_tiles * k_chunks
+
+    def cta_range(c):
+        return begin(U, TW, c * W), begin(U, TW, min((c + 1) * W, TW))
+
+    def cta_slot(c, tile):
+        _, uc1 = cta_range(c)
+        return ("slot", c * W + (0 if tile == (uc1 - 1) // k_chunks else 1), 1)
+
+    writes, epilogues, finishes = {}, {}, []
+
+    def write(loc, tile, gw):
+        assert loc not in writes, f"{loc} written twice"
+        writes[loc] = (tile, gw)
+
+    for gw in range(TW):
+        c = gw // W
+        uc, uc1 = cta_range(c)
+        u0, u1 = begin(U, TW, gw), begin(U, TW, gw + 1)
+        for tile in sorted({u // k_chunks for u in range(u0, u1)}):
+            ts, te = tile * k_chunks, (tile + 1) * k_chunks
+            a, b = max(ts, uc), min(te, uc1)
+            alone = a >= u0 and b <= u1
+            if alone and ts >= uc and te <= uc1:
+                epilogues[tile] = epilogues.get(tile, 0) + 1
+            elif u1 > b:                       # leaves the tile in mid-range
+                ps = tile - uc // k_chunks     # its slot in the CTA's shared-memory pool
+                if alone:
+                    write(cta_slot(c, tile), tile, gw)
+                elif ps < POOL:
+                    write(("pool", c, ps), tile, gw)
+                else:
+                    write(("slot", gw, 0), tile, gw)
+            else:                              # its range ends in the tile
+                write(("ring", gw), tile, gw)
+                whi = owner(U, TW, b - 1)
+                fin = whi - 1 if begin(U, TW, whi + 1) > b else whi
+                if gw != fin:
+                    continue
+                wlo = owner(U, TW, a)
+                reads, waits = [], []
+                for v in range(wlo, whi + 1):
+                    if v == whi and begin(U, TW, whi + 1) > b:
+                        ps = tile - uc // k_chunks
+                        reads.append(("pool", c, ps) if ps < POOL else ("slot", whi, 0))
+                    else:
+                        reads.append(("ring", v))
+                        if v != gw:
+                            waits.append(v)              # its shared-memory flag
+                clo, chi = owner(U, TW, ts) // W, owner(U, TW, te - 1) // W
+                if clo != chi and c != clo:
+                    write(cta_slot(c, tile), tile, gw)
+                else:
+                    if clo != chi:
+                        reads += [cta_slot(cc, tile) for cc in range(clo + 1, chi + 1)]
+                    epilogues[tile] = epilogues.get(tile, 0) + 1
+                finishes.append((tile, gw, reads, waits))
+    return U, writes, epilogues, finishes
+
+
+@pytest.mark.parametrize("n_tiles,k_chunks,TW,W,POOL", [c[:4] + (p,) for c in itertools.product(
+    [1, 3, 8, 80, 160, 480], [1, 2, 8, 40, 80, 272], [8, 64, 1184, 2368], [16, 12, 8]) for p in (0, 2, 8)])
+def test_designated_finisher_plan(n_tiles, k_chunks, TW, W, POOL):
+    U = n_tiles * k_chunks
+    ctas = min(-(-U // W), max(1, TW // W))
+    TW = min(ctas * W, U)
+    U, writes, epilogues, finishes = _combine_plan(n_tiles, k_chunks, TW, W, POOL)
+    # every tile is finished exactly once
+    assert sorted(epilogues) == list(range(n_tiles)) and all(n == 1 for n in epilogues.values()), epilogues
+    for tile, gw, reads, waits in finishes:
+        for loc in reads:
+            assert loc in writes and writes[loc][0] == tile, (tile, gw, loc)
+        # a finisher waits only for warps whose range ends in the tile and that finish nothing themselves
+        for v in waits:
+            assert writes.get(("ring", v)) == (tile, v)
+            assert all(f[1] != v for f in finishes)
+    # every partial published in the workspace is read by exactly one finisher
+    readers = {}
+    for tile, gw, reads, _ in finishes:
+        for loc in reads:
+            readers[loc] = readers.get(loc, 0) + 1
+    for loc, (tile, gw) in writes.items():
+        if loc[0] in ("slot", "pool"):
+            assert readers.get(loc) == 1, (loc, tile, gw)
+        if loc[0] == "slot":
+            assert loc[1] < -(-TW // W) * W    # inside the grid's slots
+        if loc[0] == "pool":
+            assert 0 <= loc[2] < POOL
