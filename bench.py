@@ -33,6 +33,7 @@ if ROOT not in sys.path:
 METRIC = "NVFP4 decode GEMM HBM GB/s and % of B200 peak at M=1..8; full round ms"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # the B200's nominal HBM3e bandwidth (~8 TB/s), a second denominator
 KERNEL_SOURCES = ["gemm.cu", "dequant.cuh", "layout.cuh", "async.cuh"]
 
 
@@ -49,7 +50,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="only warm-up and timed replays (for an ncu launch list)")
-    ap.add_argument("--gemm-case", default=None, choices=["head", "proj", "gateup", "down"],
+    ap.add_argument("--gemm-case", default=None, choices=["head", "proj", "qkv", "gateup", "down"],
                     help="only three direct calls of one workload GEMM at --width (for an ncu capture)")
     ap.add_argument("--topk-case", type=int, default=None,
                     help="only three top-k calls with this k over --width rows of 151,936 logits (for an ncu capture)")
@@ -373,6 +374,44 @@ def gemm_sweep(dev, hbm_peak):
     return out
 
 
+def node_split(r, stream, widths, by_width):
+    """Per node kind: the round's nodes of that kind alone, chained in one graph,
+    device time per node at each width, and that kind's share of the round."""
+    import torch
+
+    from nvfp4_weight_streaming_decode_b200 import abi
+    kinds = {}
+    for i, (name, _, _, _, _) in enumerate(r.nodes):
+        kinds.setdefault(re.sub(r"\d+$", "", name), []).append(i)
+    out = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for kind, idx in kinds.items():
+        rnd = abi.Round([r.descs[i] for i in idx], abi.NVFP4_ROUND_CHAIN)
+        reps = max(3, 200 // len(idx))
+        res = {"nodes": len(idx)}
+        for M in widths:
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    rnd.replay(M, stream)
+                e0.record(stream)
+                for _ in range(reps):
+                    rnd.replay(M, stream)
+                e1.record(stream)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps / len(idx)
+            res[f"us_per_node_M{M}"] = us
+            if by_width.get(M):
+                res[f"share_of_round_M{M}"] = us * len(idx) / (by_width[M] * 1e3)
+        rnd.close()
+        out[kind] = res
+    for M in widths:
+        if by_width.get(M):
+            out[f"sum_over_kinds_ms_M{M}"] = sum(v[f"us_per_node_M{M}"] * v["nodes"] for k, v in out.items()
+                                                  if isinstance(v, dict)) / 1e3
+            out[f"round_ms_M{M}"] = by_width[M]
+    return out
+
+
 def round_io_bytes(r, M):
     """Algorithmic activation bytes of one round: X read and outputs written, per node."""
     from nvfp4_weight_streaming_decode_b200 import abi
@@ -585,6 +624,7 @@ def run_gemm_case(args):
     dev = torch.device("cuda", 0)
     M = args.width
     shapes = {"head": (151936, 5120, synth.EXP_LOGU_M6_4), "proj": (5120, 5120, synth.EXP_UNIFORM_M4_2),
+              "qkv": (15360, 5120, synth.EXP_UNIFORM_M4_2),
               "gateup": (17408, 5120, synth.EXP_UNIFORM_M4_2), "down": (5120, 17408, synth.EXP_UNIFORM_M4_2)}
     N, K, exp = shapes[args.gemm_case]
     m = make_matrix(3, 0, N, K, dev, exp)
@@ -671,17 +711,17 @@ def run_ours(args):
             rnd.replay(M, stream)
     torch.cuda.synchronize()
 
-    # per-width round times (detail): 20 replays each, an event after every replay
-    # for the median and p90 beside the mean
+    # per-width round times (detail): 20 warm-up replays, then 100 timed, an event
+    # after every replay for the median and p90 beside the mean
     by_width, p50_by_width, p90_by_width = {}, {}, {}
     if args.profile:
         args.no_sweep = args.no_cpu_baseline = True
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_rep = 20
+    n_warm_detail, n_rep = 20, 100
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_rep + 1)]
     for m in (range(1, 9) if not args.profile else ()):
         with torch.cuda.stream(stream):
-            for _ in range(3):
+            for _ in range(n_warm_detail):
                 rnd.replay(m, stream)
             evs[0].record(stream)
             for j in range(n_rep):
@@ -692,6 +732,23 @@ def run_ours(args):
         by_width[m] = evs[0].elapsed_time(evs[-1]) / n_rep
         p50_by_width[m] = statistics.median(per)
         p90_by_width[m] = percentile(per, 90)
+
+    # host submission cost of one replay: host wall time around the C-ABI call that
+    # launches the width's graph (through the Python binding), for 30 replays queued
+    # back to back; its share of the round's device time (the pages' 2.2 %)
+    submit = None
+    if not args.profile:
+        torch.cuda.synchronize()
+        host_ns = []
+        with torch.cuda.stream(stream):
+            for _ in range(30):
+                t0 = time.perf_counter_ns()
+                rnd.replay(M, stream)
+                host_ns.append(time.perf_counter_ns() - t0)
+        torch.cuda.synchronize()
+        med_us = statistics.median(host_ns) / 1e3
+        submit = {"host_us_per_replay_p50": med_us, "host_us_per_replay_max": max(host_ns) / 1e3,
+                  "share_of_round": med_us / (by_width.get(M, 0) * 1e3) if by_width.get(M) else None}
 
     # the timed region: K replays at width M
     clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
@@ -737,7 +794,7 @@ def run_ours(args):
     achieved = per_launch_bytes / per_launch_s / 1e9
     traffic_round = profiled_traffic()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak,
+                "frac": achieved / hbm_peak, "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                 "traffic": (traffic_round / launches) if traffic_round else None,
                 "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
@@ -757,6 +814,13 @@ def run_ours(args):
         rnd.replay(8, stream)
         torch.cuda.synchronize()
         topk = topk_detail(r.bufs["logits"], dev, hbm_peak)
+
+    # device-time split of the round by node kind: each kind's nodes of this round
+    # alone, chained in their own graph (same matrices and buffers), timed at width M
+    # and at width 1; the sum over kinds set against the live round
+    split = None
+    if rank == 0 and not args.no_sweep:
+        split = node_split(r, stream, (1, M), by_width)
 
     sweep = None
     verify = None
@@ -783,6 +847,8 @@ def run_ours(args):
             "round_ms_by_width": by_width,
             "round_GBps_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 for m, t in by_width.items()},
             "round_frac_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 / hbm_peak for m, t in by_width.items()},
+            "round_frac_of_nominal_by_width": {m: weight_bytes / (t * 1e-3) / 1e9 / NOMINAL_HBM_GBS
+                                               for m, t in by_width.items()},
             "round_ms_p50_by_width": p50_by_width,
             "round_ms_p90_by_width": p90_by_width,
             "read_peak": read_peak,
@@ -792,6 +858,8 @@ def run_ours(args):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x_host.numel() * 2,
                     "d2h_bytes_per_step": y_host.numel() * 4, "ms_per_step": e2e_s * 1e3 / e2e_steps},
             "gpu_launches": graph_nodes * args.steps,
+            "submission": submit,
+            "node_split": split,
             "clocks": clk,
             "gemm_sweep": sweep,
             "topk": topk,
