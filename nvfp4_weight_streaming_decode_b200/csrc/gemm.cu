@@ -16,15 +16,19 @@
 // stages with 1-D bulk copies (the TMA engine, no tensor map, no multicast),
 // one mbarrier per stage, dequantises in registers and feeds bf16 m16n8k16
 // tensor-core MMAs with the lanes of X as the 8-wide N side.  A tile
-// (32 rows) that straddles warp ranges is finished by whichever of its
-// contributors arrives last, in two levels (finish_tile): the contributors
-// inside one CTA count in at a shared-memory counter and the last of them adds
-// their partial sums in warp order; a tile that spans CTAs then has each CTA's
-// sum counted in at a global counter, and the last CTA adds them in CTA order.
-// Both orders are fixed, so results are bit-identical run to run.  In the
-// plain and fused kernels no thread ever waits on another warp or CTA; the
-// persistent round kernel at the end of the file is the one place where the
-// grid meets, at a bounded barrier between nodes.
+// (32 rows) that straddles warp ranges is combined in two levels: inside a
+// CTA, each contributing warp leaves its partial sums in shared memory and
+// raises a flag; across CTAs, each later CTA's designated warp writes its
+// CTA's sum into a workspace slot as 64-bit words carrying a ready bit.  One
+// warp -- the last range-end contributor of the CTA that holds the tile's
+// first unit -- waits (bounded) on those flags and words and adds them in warp
+// order, then CTA order (finish_tile).  A later CTA's designated warp waits
+// only on its own CTA's contributors, and those publish without waiting, so
+// the waits form no cycle.  The fused gate/up kernel keeps a one-level last-arriver
+// combine through a global counter (tile_done_global) and never waits.  Both
+// orders are fixed, so results are bit-identical run to run.  The persistent
+// round kernel at the end of the file also meets the whole grid at a bounded
+// barrier between nodes.
 //
 // PDL: every kernel signals its dependents at entry, issues its weight
 // copies (which depend on nothing), and only then waits for the preceding
