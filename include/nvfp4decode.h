@@ -104,8 +104,11 @@ NVFP4_API int nvfp4_pack_check(const uint8_t* wq_canon, const uint8_t* ws_canon,
  * verified in the same pass).  Widths 9..32 run on the decode kernel with
  * two to four blocks of 8 lanes sharing each dequantised word; widths 33..64
  * run on the tensor-memory kernel (its own per-device workspace, allocated by
- * its first call under the same capture rule; nvfp4_verify_geometry
- * describes its work split).  Other M: NVFP4_ERR_M.
+ * its first call under the same capture rule, and a buffer for X in the
+ * MMA's order sized for K up to 65,536 at first; a call with a longer K than
+ * any before grows it, synchronising the device, under the same rule;
+ * nvfp4_verify_geometry describes its work split).  Those widths launch two
+ * kernels: X's reordering, then the GEMM.  Other M: NVFP4_ERR_M.
  */
 NVFP4_API int nvfp4_gemm_decode(const void* X, int M, const uint8_t* wq_dev, const uint8_t* ws_dev,
                       float gscale, float* Y, int64_t N, int64_t K, nvfp4_stream_t stream);
@@ -325,8 +328,9 @@ NVFP4_API int nvfp4_gemm_grouped(const void* X, int x_per_route, const int32_t* 
 /*
  * Host helper (no GPU needed): the work split nvfp4_gemm_decode uses at a
  * verify width M (9..64) on a device with `sm_count` SMs -- `ctas` CTAs,
- * each owning a contiguous range of the `units` (512-row tile group, 64-column
- * chunk) units -- and `nl`, the MMA's N (M padded to a multiple of 16).
+ * each owning a contiguous range of the `units` (256-row group, pair of
+ * 64-column chunks) units -- and `nl`, the MMA's N (M padded to a multiple
+ * of 16).
  * Returns NVFP4_ERR_M / NVFP4_ERR_SHAPE exactly when the call would.
  */
 NVFP4_API int nvfp4_verify_geometry(int M, int64_t N, int64_t K, int sm_count, int64_t* ctas, int64_t* units,
@@ -359,10 +363,11 @@ NVFP4_API int nvfp4_last_cuda_error(void);
  * bounded waits, else an OR of these flags:
  *    1  decode GEMM: a warp's bulk-copy ring wait gave up
  *    2  persistent round: the grid barrier between nodes gave up
- *    4  decode GEMM: the split-K gather's copy wait gave up (sums then read
- *       from global memory)
- *    8  verify widths (33..64): a streaming warp's wait gave up
- *   16  verify widths (33..64): the MMA thread's wait gave up
+ *    4  decode GEMM: a split-K combine wait gave up -- a gather copy (sums
+ *       then read from global memory) or a finisher's wait on a partial
+ *       (that tile's Y is wrong)
+ *    8  verify widths (33..64): a dequantisation warp's wait gave up
+ *   16  verify widths (33..64): the MMA or X-staging thread's wait gave up
  *   32  grouped experts: a route named an expert outside 0..E-1 or with
  *       misaligned planes (its rows are zero)
  *   64  grouped experts: a bounded wait gave up

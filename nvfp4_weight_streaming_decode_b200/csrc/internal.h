@@ -83,7 +83,7 @@ cudaError_t noalloc_clear_scratch();
 // tensor-memory path: geometry of a call, its launch, and its status word.
 constexpr int kVerifyMinM = 9, kVerifyMaxM = 64;
 struct VerifyGeometry {
-    long long n_tiles32, n_groups, k_chunks, units, ctas;
+    long long n_tiles32, n_groups, k_chunks, k_pairs, units, ctas;
     int nl, tmem_cols;
 };
 int verify_geometry(int M, int64_t N, int64_t K, int sm_count, VerifyGeometry* g);

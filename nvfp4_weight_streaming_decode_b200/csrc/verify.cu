@@ -11,25 +11,32 @@
 // At these widths the product no longer fits the register MMA path, so the
 // multiply runs on the fifth-generation tensor cores (tcgen05) with both the
 // accumulators and the A operand in tensor memory:
-//   * A CTA (one per SM) owns a contiguous range of (512-row tile group,
-//     64-column chunk) units -- stream-K at CTA granularity -- so every SM
-//     gets the same number of weight bytes, whatever the shape.
-//   * Sixteen dequantisation warps each stream one 32-row tile of the group
-//     through their own ring of 1-D bulk copies, dequantise it exactly (the
-//     same bit placement and bf16 scale multiply as the decode kernel) and
-//     store it as bf16 into tensor memory with one tcgen05.st per row group:
-//     the 16x256b store shape takes the m16n8k16 A fragment as it stands,
-//     so the MMA's k order is the fragment's (per step s, k = 4t + j is the
-//     chunk's column 16t + 4s + j).  They also stage the chunk of X (the
-//     MMA's N side, M rows padded to a multiple of 16) in shared memory in
-//     that k order.  A and X are double-buffered; keeping A out of shared
-//     memory leaves its bandwidth to the weight ring and X.
-//   * One thread of a seventeenth warp issues tcgen05.mma (M = 128, N =
-//     16..64, K = 16; four per tile and chunk) into four accumulators in
-//     tensor memory and commits each chunk to an mbarrier that frees its
-//     buffers.  (The commit latency is paid once per chunk, so the more rows
-//     a chunk carries, the less of it shows.)
-//   * At the end of a tile group's K range the dequantisation warps read the
+//   * A first kernel (verify_xprep_kernel) writes X once per call in the
+//     MMA's operand order (K-major 8 x 16-byte core matrices, the columns of
+//     each 64-column chunk permuted to the order in which the dequantised
+//     words reach tensor memory), so a CTA stages a hand-off's X with one
+//     1-D bulk copy.
+//   * A CTA (one per SM) owns a contiguous range of (256-row group, pair of
+//     64-column chunks) units -- stream-K at CTA granularity -- so every SM
+//     gets the same number of weight bytes, whatever the shape.  A unit is
+//     one hand-off to the tensor cores.
+//   * Eight dequantisation warps each stream one 32-row slice of the group
+//     through their own ring of 1-D bulk copies (both units of a hand-off per
+//     stage), read the next hand-off's codes while they dequantise this one
+//     exactly (the same bit placement and bf16 scale multiply as the decode
+//     kernel), and store it as bf16 into tensor memory with one tcgen05.st
+//     per unit and row group: the 16x256b store shape takes the m16n8k16 A
+//     fragment as it stands.
+//   * Hand-offs rotate through three buffers: A in tensor memory, X in shared
+//     memory.  Buffer b's full barrier takes the eight warps' arrivals and
+//     X's bytes (one thread of an eleventh warp copies X); its free barrier
+//     takes the commits of the MMAs that read it.
+//   * Two issuing threads, one per 128-row tile and on two sub-partitions
+//     (the issue competes with the dequantisation there), each wait for a
+//     full buffer and issue tcgen05.mma (M = 128, N = 16..64, K = 16; eight
+//     per tile and hand-off) into the tile's accumulator in tensor memory,
+//     then commit to the buffer's free barrier.
+//   * At the end of a group's K range the dequantisation warps read the
 //     accumulators back (tcgen05.ld) and write Y, or, for a group split
 //     between CTAs, a partial sum; the last CTA to finish a split group adds
 //     the partials in CTA order (deterministic) and writes Y.
@@ -52,50 +59,65 @@ __device__ unsigned int g_verify_status;
 
 namespace {
 
-constexpr int kVTiles = 4;                     // 128-row tiles per CTA group (512 rows)
-constexpr int kVWarps = 4 * kVTiles;           // dequantisation warps: one per 32-row tile
-constexpr int kVCtasPerSM = 1;                 // one CTA per SM: shared memory holds its operands
-constexpr int kVBufs = 2;                      // operand (A, X) buffers: chunks in flight to the tensor cores
-constexpr int kVThreads = (kVWarps + 1) * 32;  // + the MMA / tensor-memory warp
-constexpr int kVStages = 6;                    // per-warp ring depth, one unit per stage
-constexpr int kVTileRows = 128;                // MMA M
-constexpr int kVMaxNL = 64;                    // MMA N at most (M rows of X, padded to 16)
-constexpr int kXBytes = kVMaxNL * kChunkK * 2;     // one chunk of X: 8 KB
-static_assert(kVMaxNL * 8 <= kVWarps * 32, "each dequantisation thread stages at most one 16-byte piece of X");
-// Tensor memory (512 columns): accumulators in columns [0, 4 * nl) (nl <= 64),
-// the bf16 A operand from column 256: per buffer and tile, 128 lanes x 32
-// columns (a chunk's 64 values per row, two per column).
+constexpr int kVTiles = 2;                       // 128-row MMA tiles per group (256 rows)
+constexpr int kVSlices = 4 * kVTiles;            // 32-row slices per group
+constexpr int kVPair = 2;                        // 64-column chunks per hand-off
+#ifndef NVFP4_VSPLIT
+#define NVFP4_VSPLIT 1
+#endif
+constexpr int kVSplit = NVFP4_VSPLIT;            // dequantisation warps per slice, each on its share of the chunks
+constexpr int kVWarps = kVSlices * kVSplit;
+constexpr int kVUPW = kVPair / kVSplit;          // units per warp and hand-off
+static_assert(kVPair % kVSplit == 0, "the chunks of a hand-off divide among a slice's warps");
+constexpr int kVBufs = 3;                        // hand-offs in flight: A buffers (tensor memory), X buffers (shared)
+constexpr int kVStages = 7;                      // per-warp ring depth, one hand-off per stage
+constexpr int kVMmaWarp = kVWarps;               // one thread per tile issues its MMAs (warps kVWarps..)
+constexpr int kVXWarp = kVWarps + kVTiles;       // one thread stages X
+constexpr int kVThreads = (kVXWarp + 1) * 32;
+constexpr int kVCtasPerSM = 1;                   // one CTA per SM: it holds all 512 tensor-memory columns
+constexpr int kVTileRows = 128;                  // MMA M
+constexpr int kVMaxNL = 64;                      // MMA N at most (M rows of X, padded to 16)
+constexpr int kVGroupRows = kVTiles * kVTileRows;        // 256
+constexpr int kVStageBytes = kVUPW * kUnitBytes;         // codes of the warp's units, then their scales
+constexpr int kXChunkBytes = kVMaxNL * kChunkK * 2;      // one chunk of X at NL = 64: 8 KB
+constexpr int kXBufBytes = kVPair * kXChunkBytes;        // 16 KB
+// Tensor memory (512 columns): accumulators in columns [0, kVTiles * nl)
+// (nl <= 64); the bf16 A operand from column 128: per buffer and tile, 128
+// lanes x 64 columns (a hand-off's 128 values per row, two per column).
 constexpr int kVTmemCols = 512;
-constexpr int kATmemCol = kVTiles * kVMaxNL;       // 256
-constexpr int kATmemTileCols = kChunkK / 2;        // 32
-constexpr int kVGroupRows = kVTiles * kVTileRows;  // 512
-constexpr int kVSlotFloats = kVMaxNL * kVGroupRows;  // a partial: [512 rows][64 m] floats
-constexpr int kVMaxGroups = 1 << 16;                // tile groups a call may have
-constexpr int kVMaxSplit = 4;                      // CTAs per tile group at most, on average
+constexpr int kATmemCol = kVTiles * kVMaxNL;             // 128
+constexpr int kATmemTileCols = kVPair * kChunkK / 2;     // 64
+static_assert(kATmemCol + kVBufs * kVTiles * kATmemTileCols <= kVTmemCols, "tensor memory holds A and D");
+static_assert(kVSlices * 32 == kVGroupRows, "one dequantisation thread per row of a group and warp share");
+constexpr int kVSlotFloats = kVMaxNL * kVGroupRows;      // a partial: [256 rows][64 m] floats
+constexpr int kVMaxGroups = 1 << 16;                     // groups a call may have
+constexpr int kVMaxSplit = 8;                            // CTAs per group at most, on average
+constexpr int kFinBatch = kVSplit == 1 ? 4 : 2;          // contributors' partials in flight in the final sum
 
 // shared-memory map (bytes)
-constexpr int kOffX = 0;                                   // [kVBufs buffers][8 KB]
-constexpr int kOffRing = kOffX + kVBufs * kXBytes;         // [kVWarps warps][kVStages stages][1152 B]
-constexpr int kOffBar = kOffRing + kVWarps * kVStages * kUnitBytes;
-// barriers: ring[8][3], full[2], empty[2], acc, acc_free, part_done, last_ready, fin
-constexpr int kBarRing = 0, kBarFull = kVWarps * kVStages, kBarEmpty = kBarFull + kVBufs, kBarAcc = kBarEmpty + kVBufs,
-              kBarAccFree = kBarAcc + 1, kBarPart = kBarAccFree + 1, kBarLast = kBarPart + 1,
-              kBarFin = kBarLast + 1, kNumBars = kBarFin + 1;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;            // tmem base, abort, last, pad
+constexpr int kOffX = 0;                                          // [kVBufs][16 KB]
+constexpr int kOffRing = kOffX + kVBufs * kXBufBytes;             // [kVWarps][kVStages][kVStageBytes]
+constexpr int kOffBar = kOffRing + kVWarps * kVStages * kVStageBytes;
+// full[b]: the dequantisation warps' arrivals and X's bytes for the hand-off in buffer b;
+// free[b]: the MMAs that read buffer b are done (one commit)
+constexpr int kBarRing = 0, kBarFull = kVWarps * kVStages, kBarFree = kBarFull + kVBufs, kBarAcc = kBarFree + kVBufs,
+              kBarPart = kBarAcc + 1, kBarLast = kBarPart + 1, kBarFin = kBarLast + 1, kNumBars = kBarFin + 1;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;                  // tmem base, abort, last, pad
 constexpr int kVSmemBytes = kOffMisc + 16;
+static_assert(kVSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 struct VParams {
     const uint8_t* wq;
     const uint8_t* ws;
-    const uint16_t* X;
+    const uint8_t* Xp;   // X in the MMA's order: [chunk][nl / 8][8 octets][8 rows][16 B]
     float* Y;
-    float* part;         // [ctas][2 slots][64][256]
+    float* part;         // [ctas][2 slots][256 rows][64]
     unsigned* counters;  // [groups]
     float gscale;
     int M, NL, tmem_cols;
-    long long N, K;
-    int KC, n_tiles32, n_groups;
-    long long units, ctas;  // stream-K over units = n_groups * KC
+    long long N;
+    int KC, KP, n_tiles32, n_groups;  // chunks, chunk pairs, 32-row tiles, groups
+    long long units, ctas;            // stream-K over units = n_groups * KP
     uint32_t idesc;
 };
 
@@ -108,6 +130,13 @@ __device__ __forceinline__ long long vrange_owner(long long units, long long t, 
     return ((x + 1) * t - 1) / units;
 }
 
+__device__ __forceinline__ uint64_t evict_last_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // K-major operand in shared memory without swizzle: 8-row core matrices of
 // 16-byte rows; the two k-octets of one K = 16 step are 128 bytes apart
 // (leading byte offset) and consecutive 8-row groups 1024 bytes apart
@@ -117,16 +146,6 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr)
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(1024u >> 4) << 32) |
            ((uint64_t)1 << 46);  // descriptor version for this architecture; no swizzle, base offset 0
 }
-__device__ __forceinline__ uint32_t kmajor_off(int row, int octet)
-{
-    return (uint32_t)((row >> 3) * 1024 + octet * 128 + (row & 7) * 16);
-}
-
-__device__ __forceinline__ void st_shared_v2(uint32_t a, uint32_t x, uint32_t y)
-{
-    asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(a), "r"(x), "r"(y) : "memory");
-}
-
 // 16 lanes x 4 x 256 bits of this warp's lane quarter from registers: register
 // 4i + j goes to lane (taddr's lane) + (t / 4) + 8 * (j / 2), column (taddr's
 // column) + 8i + 2 * (t % 4) + (j % 2), for thread t -- the layout of the
@@ -180,9 +199,24 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16])
 constexpr uint32_t kVSleepNs = 1000;
 constexpr uint32_t kVWaitLimit = 1u << 20;
 
+// Non-blocking test of a phase (cheaper than try_wait when it has completed,
+// the common case for the ring and buffer waits).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait of a whole warp that also gives up once the CTA aborted.
 __device__ __forceinline__ bool vwait(uint32_t bar, uint32_t parity, const volatile int* abort)
 {
+    if (__all_sync(0xffffffffu, mbar_test(bar, parity))) return true;
     for (uint32_t it = 0; it < kVWaitLimit; ++it) {
         if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, kVSleepNs))) return true;
         if (*abort) return false;
@@ -193,6 +227,7 @@ __device__ __forceinline__ bool vwait(uint32_t bar, uint32_t parity, const volat
 // The same for one thread.
 __device__ __forceinline__ bool vwait1(uint32_t bar, uint32_t parity, const volatile int* abort)
 {
+    if (mbar_test(bar, parity)) return true;
     for (uint32_t it = 0; it < kVWaitLimit; ++it) {
         if (mbar_try_wait_sleep(bar, parity, kVSleepNs)) return true;
         if (*abort) return false;
@@ -206,6 +241,36 @@ __device__ __forceinline__ void vabort(volatile int* abort, unsigned bit)
     atomicOr(&g_verify_status, bit);
 }
 
+// X in the MMA's operand order, once per call: Xp[c] is chunk c (columns
+// 64c..64c+63) as nl / 8 groups of 8 rows, each group 8 k-octets of 8 rows x
+// 16 bytes (the K-major core matrices of kmajor_desc).  MMA step s of a chunk
+// takes as its k = 4t + j (t, j = 0..3) the chunk's column 16t + 4s + j --
+// the order in which the dequantised words reach tensor memory -- so octet
+// 2s + h holds columns 32h + 4s + (0..3) and 32h + 16 + 4s + (0..3).  Rows
+// past M and columns past K are zero.  One thread per 16-byte piece.
+__global__ void __launch_bounds__(256) verify_xprep_kernel(const uint16_t* __restrict__ X, uint8_t* __restrict__ Xp,
+                                                           int M, int NL, long long K, long long pieces)
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // X comes from the preceding kernel, and the preceding verify kernel may still read Xp
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (i >= pieces) return;
+    const int r8 = (int)(i & 7), o = (int)((i >> 3) & 7);
+    const long long rest = i >> 6;
+    const int groups8 = NL >> 3;
+    const int row = (int)(rest % groups8) * 8 + r8;
+    const long long c = rest / groups8;
+    uint2 lo = make_uint2(0u, 0u), hi = make_uint2(0u, 0u);
+    if (row < M) {
+        const long long col = c * kChunkK + 32 * (o & 1) + 4 * (o >> 1);
+        const uint16_t* src = X + (long long)row * K + col;
+        if (col < K) lo = *reinterpret_cast<const uint2*>(src);  // K % 16 == 0: all four columns exist
+        if (col + 16 < K) hi = *reinterpret_cast<const uint2*>(src + 16);
+    }
+    *reinterpret_cast<uint4*>(Xp + i * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+}
+
 __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VParams p)
 {
     extern __shared__ __align__(1024) uint8_t vsm[];
@@ -214,21 +279,28 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
     const uint32_t bars = base + kOffBar;
     volatile int* misc = reinterpret_cast<volatile int*>(vsm + kOffMisc);  // [0] tmem base [1] abort [2] last
     volatile int* abort = misc + 1;
-    const long long U = p.units, T = p.ctas, KC = p.KC;
+    const long long U = p.units, T = p.ctas;
+    const int KC = p.KC, KP = p.KP;
     const long long cta = blockIdx.x;
     const long long u0 = vrange_begin(U, T, cta), u1 = vrange_begin(U, T, cta + 1);
-    const int n = (int)(u1 - u0);  // this CTA's (group, chunk) units; >= 1 as ctas <= units
+    const int n = (int)(u1 - u0);  // this CTA's (group, chunk pair) units; >= 1 as ctas <= units
+    const long long group0 = u0 / KP;
+    const int pr0 = (int)(u0 - group0 * KP);
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
-            const bool per_warp = (i >= kBarFull && i < kBarFull + kVBufs) || i == kBarAccFree || i == kBarPart;
-            mbar_init(bars + 8 * i, per_warp ? (uint32_t)kVWarps : 1u);
+            const bool full = i >= kBarFull && i < kBarFull + kVBufs;
+            const bool per_issuer = (i >= kBarFree && i < kBarFree + kVBufs) || i == kBarAcc || i == kBarFin;
+            mbar_init(bars + 8 * i, full ? (uint32_t)(kVWarps + 1)
+                                    : i == kBarPart ? (uint32_t)kVWarps
+                                    : per_issuer    ? (uint32_t)kVTiles
+                                                    : 1u);
         }
         misc[1] = 0;
         misc[2] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == kVWarps) {
+    if (warp == kVMmaWarp) {
         // tensor memory for the accumulators and the A operand (all 512 columns)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(base + kOffMisc),
                      "r"(p.tmem_cols)
@@ -243,157 +315,176 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
 
     if (warp < kVWarps) {
         const int w = warp;
-        const uint8_t* ring = vsm + kOffRing + w * (kVStages * kUnitBytes);
-        const uint32_t ring_s = base + kOffRing + w * (kVStages * kUnitBytes);
+        const int slice = w % kVSlices;        // this warp's 32 rows of the group
+        const int h0 = (w / kVSlices) * kVUPW;  // and its first chunk of each pair
+        const uint8_t* ring = vsm + kOffRing + w * (kVStages * kVStageBytes);
+        const uint32_t ring_s = base + kOffRing + w * (kVStages * kVStageBytes);
         const uint32_t rbar = bars + 8 * (kBarRing + w * kVStages);
         const uint64_t pol = evict_first_policy();
-        // stage j <-> unit x = u0 + j: this warp's 32-row tile of that unit's group, one chunk
-        auto tile_ok = [&](int j) { return ((u0 + j) / KC) * kVWarps + w < p.n_tiles32; };
-        // (group, chunk) of unit u0 once; every later position advances incrementally
-        const long long group0 = u0 / KC;
-        const int c0 = (int)(u0 - group0 * KC);
+        // Stage j <-> unit u0 + j: this warp's slice of that unit's group, chunks
+        // 2 pr + h0 .. + kVUPW - 1 of its pair pr that exist; the units it copies.
+        auto stage_units = [&](long long x) {
+            const long long g = x / KP;
+            const int c0 = 2 * (int)(x - g * KP) + h0;
+            const int nw = KC - c0 < kVUPW ? KC - c0 : kVUPW;
+            return (g * kVSlices + slice < p.n_tiles32 && nw > 0) ? nw : 0;
+        };
         long long igroup = group0;  // the next stage to issue (lane 0), in stage order
-        int ic = c0;
+        int ipr = pr0;
         auto issue = [&](int j) {  // lane 0; called for j = 0, 1, 2, ... in order
-            const long long t32 = igroup * kVWarps + w;
-            const long long unit = t32 * KC + ic;
-            if (++ic == (int)KC) {
-                ic = 0;
+            const long long t32 = igroup * kVSlices + slice;
+            const int c0 = 2 * ipr + h0;
+            if (++ipr == KP) {
+                ipr = 0;
                 ++igroup;
             }
-            if (t32 >= p.n_tiles32) return;  // rows past N: no data, zeros below
+            const int nw = KC - c0 < kVUPW ? KC - c0 : kVUPW;
+            if (t32 >= p.n_tiles32 || nw <= 0) return;  // rows past N, chunks past K: no data
+            const long long unit = t32 * KC + c0;  // a slice's units of one pair are consecutive
             const int slot = j % kVStages;
             const uint32_t bar = rbar + 8 * slot;
-            mbar_expect_tx(bar, (uint32_t)kUnitBytes);
-            bulk_load(ring_s + slot * kUnitBytes, p.wq + unit * kUnitQ, kUnitQ, bar, pol);
-            bulk_load(ring_s + slot * kUnitBytes + kUnitQ, p.ws + unit * kUnitS, kUnitS, bar, pol);
+            mbar_expect_tx(bar, (uint32_t)(nw * kUnitBytes));
+            bulk_load(ring_s + slot * kVStageBytes, p.wq + unit * kUnitQ, (uint32_t)(nw * kUnitQ), bar, pol);
+            bulk_load(ring_s + slot * kVStageBytes + kVUPW * kUnitQ, p.ws + unit * kUnitS, (uint32_t)(nw * kUnitS),
+                      bar, pol);
         };
         if (lane == 0) {
             const int npre = n < kVStages ? n : kVStages;
             for (int j = 0; j < npre; ++j) issue(j);
         }
-        // X and the outputs come from / go to the previous kernel's buffers
+        // the outputs and the workspace are the previous kernels' until they are done
         asm volatile("griddepcontrol.wait;" ::: "memory");
 
-        // X pieces of this thread: piece pc = 16 bytes of row pc / 8, columns 8 (pc % 8)
-        // .. +7 of a chunk (nl <= 64 rows: at most one piece per thread, 512 threads).
-        // In the MMA's k order step s takes, as k = 4u + j (u = 0..3, j = 0..3), the
-        // chunk's columns 16u + 4s + j -- the order in which the dequantised words go
-        // to tensor memory -- so each 8-byte half of a piece (four columns) lands in
-        // step s's octet u / 2, at byte 8 * (u % 2).  Everything but the chunk's column
-        // and the buffer is fixed per thread, so it is worked out once here.
-        const int pc = w * 32 + lane;
-        const bool x_piece = pc < p.NL * 8;                  // this thread stages a piece
-        const int x_row = pc >> 3, x_o = pc & 7;
-        const bool x_row_ok = x_piece && x_row < p.M;        // rows past M stay zero
-        const uint16_t* x_src = p.X + (long long)(x_row_ok ? x_row : 0) * p.K + 8 * x_o;
-        uint32_t x_dst[2];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int c4 = 8 * x_o + 4 * half;  // first of the four columns
-            const int u = c4 >> 4, st = (c4 >> 2) & 3;
-            x_dst[half] = kmajor_off(x_piece ? x_row : 0, 2 * st + (u >> 1)) + 8 * (u & 1);
-        }
-        auto load_x = [&](int cc, uint4& xr) {
-            xr = make_uint4(0u, 0u, 0u, 0u);
-            if (x_row_ok && (long long)cc * kChunkK + 8 * x_o < p.K)
-                xr = *reinterpret_cast<const uint4*>(x_src + (long long)cc * kChunkK);
-        };
-        auto store_x = [&](int bb, const uint4& xr) {
-            if (x_piece) {
-                const uint32_t xb = base + kOffX + bb * kXBytes;
-                st_shared_v2(xb + x_dst[0], xr.x, xr.y);
-                st_shared_v2(xb + x_dst[1], xr.z, xr.w);
-            }
-        };
-        // X of the first chunk goes straight into buffer 0; every later chunk's X is
-        // loaded at the top of the iteration before it and stored at that iteration's
-        // end, once its buffer is free (the loads have landed by then).
-        uint4 xr;
-        load_x(c0, xr);
-        store_x(0, xr);
-        const int trow = 32 * (w & 3);  // first row of this warp in its 128-row tile
-        const int tt = w >> 2;          // which tile of the group
+        const int trow = 32 * (slice & 3);  // first row of this warp in its 128-row tile
+        const int tt = slice >> 2;          // which tile of the group
         int seg = 0, split = 0;
-        int pend_lo = n, pend_hi = n;   // ring stages issued but not consumed, for the abort drain
-        long long group = group0;
-        int c = c0;
-        for (int j = 0; j < n; ++j) {
-            const long long t32 = group * kVWarps + w;
-            const bool valid = t32 < p.n_tiles32;
-            const int slot = j % kVStages;
-            if (j + 1 < n) load_x(c + 1 == (int)KC ? 0 : c + 1, xr);  // stored into the next buffer at this iteration's end
-            uint32_t q[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            uint32_t sw = 0u;
-            if (valid) {
-                if (!vwait(rbar + 8 * slot, (uint32_t)((j / kVStages) & 1), abort)) {
-                    if (lane == 0 && !*abort) vabort(abort, 1u);
-                    pend_lo = j;
-                    pend_hi = (j + kVStages < n) ? j + kVStages : n;
-                    break;
-                }
-                const uint8_t* st = ring + slot * kUnitBytes;
-                const uint4 q0 = *reinterpret_cast<const uint4*>(st + 16 * lane);
-                const uint4 q1 = *reinterpret_cast<const uint4*>(st + 512 + 16 * lane);
-                sw = *reinterpret_cast<const uint32_t*>(st + kUnitQ + 4 * lane);
-                q[0] = q0.x; q[1] = q0.y; q[2] = q0.z; q[3] = q0.w;
-                q[4] = q1.x; q[5] = q1.y; q[6] = q1.z; q[7] = q1.w;
+        // Ring bookkeeping for the abort drain: stages [0, issued) have been issued and
+        // [0, waited) waited for, so the copies of [waited, issued) may be in flight.
+        int issued = n < kVStages ? n : kVStages, waited = 0;
+        // units this warp dequantises at (group, pair): none past N or past K
+        auto units_at = [&](long long g, int prr) {
+            const int nw0 = KC - (2 * prr + h0);
+            return g * kVSlices + slice >= p.n_tiles32 ? 0 : nw0 < kVUPW ? (nw0 > 0 ? nw0 : 0) : kVUPW;
+        };
+        // the codes and scales of stage j (ring slot rslot, phase parity rpar) into
+        // registers, after its ring wait; stages are loaded in order
+        int rslot = 0;
+        uint32_t rpar = 0;
+        auto load_stage = [&](int j, int nwj, uint32_t (&qq)[kVUPW][8], uint32_t (&ss)[kVUPW]) {
+            const int slot = rslot;
+            const uint32_t par = rpar;
+            if (++rslot == kVStages) {
+                rslot = 0;
+                rpar ^= 1u;
             }
-            const int b = j % kVBufs;  // buffer b is free: the previous iteration's end waited for it
-            // A: this warp's 32 rows of its tile for this chunk, bf16, into tensor memory
-            // (lanes = rows, two values per column).  Word s of row group r holds rows
-            // 16r+g (a[s][0], a[s][2]) and 16r+g+8 (a[s][1], a[s][3]) at columns
-            // 16t+4s+{0,1} and {2,3}: MMA step s, k = 4t + {0,1} and {2,3}, i.e. the
-            // step's columns 2t and 2t + 1.
-            const uint32_t acol = tmem + (uint32_t)(kATmemCol + (b * kVTiles + tt) * kATmemTileCols);
-            uint32_t S[2][2] = {{0u, 0u}, {0u, 0u}};
-            if (valid) scale_pairs(sw, S);
+            if (nwj > 0) {
+                if (!__all_sync(0xffffffffu, mbar_test(rbar + 8 * slot, par)) && !warp_wait(rbar + 8 * slot, par))
+                    return false;
+                const uint8_t* st = ring + slot * kVStageBytes;
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                uint32_t a[4][4];
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    if (valid) {
-                        dequant_word(q[4 * r + s], S, r, a[s]);
-                    } else {
-                        a[s][0] = a[s][1] = a[s][2] = a[s][3] = 0u;
+                for (int h = 0; h < kVUPW; ++h) {
+                    if (h < nwj) {
+                        const uint4 q0 = *reinterpret_cast<const uint4*>(st + h * kUnitQ + 16 * lane);
+                        const uint4 q1 = *reinterpret_cast<const uint4*>(st + h * kUnitQ + 512 + 16 * lane);
+                        ss[h] = *reinterpret_cast<const uint32_t*>(st + kVUPW * kUnitQ + h * kUnitS + 4 * lane);
+                        qq[h][0] = q0.x; qq[h][1] = q0.y; qq[h][2] = q0.z; qq[h][3] = q0.w;
+                        qq[h][4] = q1.x; qq[h][5] = q1.y; qq[h][6] = q1.z; qq[h][7] = q1.w;
                     }
                 }
-                const uint32_t v[16] = {a[0][0], a[0][2], a[0][1], a[0][3], a[1][0], a[1][2], a[1][1], a[1][3],
-                                        a[2][0], a[2][2], a[2][1], a[2][3], a[3][0], a[3][2], a[3][1], a[3][3]};
-                tc_st_16x256b_x4(acol + ((uint32_t)(trow + 16 * r) << 16), v);
             }
-            // the A stores are complete before the MMA thread is told
+            waited = j + 1;
+            return true;
+        };
+        long long group = group0;
+        int pr = pr0;
+        int nw = units_at(group, pr);
+        // The next hand-off's codes are read one iteration ahead: its ring wait and
+        // loads overlap this hand-off's dequantisation.
+        uint32_t q[kVUPW][8], sw[kVUPW];
+        bool ok = load_stage(0, nw, q, sw);
+        int ab = 0;         // A buffer of hand-off j: j % kVBufs
+        uint32_t apar = 0;  // (j / kVBufs) & 1: the buffer's use j - kVBufs completed phase apar ^ 1
+        for (int j = 0; ok && j < n; ++j) {
+            const long long t32 = group * kVSlices + slice;
+            long long group1 = group;
+            int pr1 = pr + 1;
+            if (pr1 == KP) {
+                pr1 = 0;
+                ++group1;
+            }
+            int nw1 = 0;
+            uint32_t q1[kVUPW][8], sw1[kVUPW];
+            if (j + 1 < n) {
+                nw1 = units_at(group1, pr1);
+                if (!load_stage(j + 1, nw1, q1, sw1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            // A buffer b was last read by the MMAs of hand-off j - kVBufs
+            const int b = ab;
+            if (j >= kVBufs && !vwait(bars + 8 * (kBarFree + b), apar ^ 1u, abort)) {
+                ok = false;
+                break;
+            }
+            if (++ab == kVBufs) {
+                ab = 0;
+                apar ^= 1u;
+            }
+            tc_fence_after();
+            if (nw > 0) {
+                // A: this warp's 32 rows of its tile for its chunks, bf16, into tensor memory
+                // (lanes = rows, two values per column).  Word s of row group r of unit h
+                // holds rows 16r+g (a[s][0], a[s][2]) and 16r+g+8 (a[s][1], a[s][3]) at
+                // columns 16t+4s+{0,1} and {2,3} of chunk h: MMA step 4h + s, k = 4t +
+                // {0,1} and {2,3}, i.e. the step's columns 2t and 2t + 1.
+                const uint32_t acol = tmem + (uint32_t)(kATmemCol + (b * kVTiles + tt) * kATmemTileCols);
+#pragma unroll
+                for (int h = 0; h < kVUPW; ++h) {
+                    if (h < nw) {
+                        uint32_t S[2][2];
+                        scale_pairs(sw[h], S);
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            uint32_t a[4][4];
+#pragma unroll
+                            for (int s = 0; s < 4; ++s) dequant_word(q[h][4 * r + s], S, r, a[s]);
+                            const uint32_t v[16] = {a[0][0], a[0][2], a[0][1], a[0][3], a[1][0], a[1][2],
+                                                    a[1][1], a[1][3], a[2][0], a[2][2], a[2][1], a[2][3],
+                                                    a[3][0], a[3][2], a[3][1], a[3][3]};
+                            tc_st_16x256b_x4(acol + (uint32_t)(32 * (h0 + h)) + ((uint32_t)(trow + 16 * r) << 16), v);
+                        }
+                    }
+                }
+            }
+            // the A stores are complete before the MMA threads are told
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
-            // The tensor cores read A and X, and the next bulk copy writes this ring
-            // slot, through the async proxy: order this warp's shared-memory accesses
-            // first.  The slot is refilled only now, after the dequantisation above
-            // consumed every word read from it.
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            // Slot j is refilled only now: every word read from it has been dequantised
+            // and stored, so the copy cannot overtake the reads.
             __syncwarp();
             if (lane == 0) {
                 if (j + kVStages < n) issue(j + kVStages);
                 mbar_arrive(bars + 8 * (kBarFull + b));
             }
+            if (j + kVStages < n) issued = j + kVStages + 1;
 
-            if (c == (int)KC - 1 || j == n - 1) {
+            if (pr == KP - 1 || j == n - 1) {
                 // end of this group's K range in this CTA: read the accumulators back
                 if (!vwait(bars + 8 * kBarAcc, (uint32_t)(seg & 1), abort)) {
-                    if (lane == 0 && !*abort) vabort(abort, 1u);
-                    pend_lo = j + 1;
-                    pend_hi = (j + 1 + kVStages < n) ? j + 1 + kVStages : n;
+                    ok = false;
                     break;
                 }
                 tc_fence_after();
-                const long long ps = group * KC;  // the group's first unit
-                const bool whole = ps >= u0 && ps + KC <= u1;
+                const long long ps = group * KP;  // the group's first unit
+                const bool whole = ps >= u0 && ps + KP <= u1;
                 const long long row_g = t32 * 32 + lane;  // output row of this thread
-                const uint32_t taddr = tmem + ((uint32_t)(32 * (w & 3)) << 16) + (uint32_t)(tt * p.NL);
+                const uint32_t taddr = tmem + ((uint32_t)trow << 16) + (uint32_t)(tt * p.NL);
                 const int pslot = ps <= u0 ? 0 : 1;  // this CTA's first or last segment
-                // a partial: this row's nl sums, contiguous ([512 rows][64] per slot)
-                float* pdst = p.part + (cta * 2 + pslot) * (long long)kVSlotFloats + (w * 32 + lane) * kVMaxNL;
-                for (int m0 = 0; m0 < p.NL; m0 += 16) {
+                // a partial: this row's nl sums, contiguous ([256 rows][64] per slot)
+                float* pdst = p.part + (cta * 2 + pslot) * (long long)kVSlotFloats + (slice * 32 + lane) * kVMaxNL;
+                // the slice's warps share the columns: blocks of 16, dealt round robin
+                for (int m0 = 16 * (w / kVSlices); m0 < p.NL; m0 += 16 * kVSplit) {
                     uint32_t v[16];
                     tc_ld16(taddr + (uint32_t)m0, v);
                     if (!whole) {
@@ -406,17 +497,18 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                             if (m0 + i < p.M) p.Y[(m0 + i) * p.N + row_g] = (__uint_as_float(v[i]) * kEpilogueScale) * p.gscale;
                     }
                 }
+                // The next group's first MMA overwrites the accumulators only after every
+                // warp's next arrival on a full barrier, which follows these loads.
                 tc_fence_before();
-                // Partials go to another CTA: each lane makes its own stores visible at GPU
-                // scope before its warp signals (one thread's release does not cover the
-                // other warps' stores still in flight).
-                if (!whole) __threadfence();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + 8 * kBarAccFree);
                 ++seg;
                 if (!whole) {
+                    // Partials go to another CTA: each lane makes its own stores visible at GPU
+                    // scope before its warp signals (one thread's release does not cover the
+                    // other warps' stores still in flight).
+                    __threadfence();
+                    __syncwarp();
                     // count the CTA in on the group; its last contributor adds every partial
-                    const long long glo = vrange_owner(U, T, ps), ghi = vrange_owner(U, T, ps + KC - 1);
+                    const long long glo = vrange_owner(U, T, ps), ghi = vrange_owner(U, T, ps + KP - 1);
                     if (lane == 0) mbar_arrive(bars + 8 * kBarPart);
                     if (w == 0) {
                         if (!vwait(bars + 8 * kBarPart, (uint32_t)(split & 1), abort)) {
@@ -432,33 +524,44 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                         }
                     }
                     if (!vwait(bars + 8 * kBarLast, (uint32_t)(split & 1), abort)) {
-                        if (lane == 0 && !*abort) vabort(abort, 1u);
-                        pend_lo = j + 1;
-                        pend_hi = (j + 1 + kVStages < n) ? j + 1 + kVStages : n;
+                        ok = false;
                         break;
                     }
                     const int last = misc[2];
                     ++split;
                     if (last) {
-                        // every contributor's partial of this row, in CTA order, 16 sums at a time
+                        // every contributor's partial of this row, in CTA order, 16 sums at a
+                        // time, four contributors' loads in flight at once
                         const int glo_slot = vrange_begin(U, T, glo) >= ps ? 0 : 1;
-                        for (int m0 = 0; m0 < p.NL; m0 += 16) {
+                        const float* rowp = p.part + (slice * 32 + lane) * kVMaxNL;
+                        for (int m0 = 16 * (w / kVSlices); m0 < p.NL; m0 += 16 * kVSplit) {
                             float sum[16];
 #pragma unroll
                             for (int i = 0; i < 16; ++i) sum[i] = 0.f;
-                            for (long long ci = glo; ci <= ghi; ++ci) {
-                                const int sl = ci == glo ? glo_slot : 0;
-                                const float4* src = reinterpret_cast<const float4*>(
-                                    p.part + (ci * 2 + sl) * (long long)kVSlotFloats + (w * 32 + lane) * kVMaxNL + m0);
-                                float4 v4[4];
+                            for (long long c0 = glo; c0 <= ghi; c0 += kFinBatch) {
+                                float4 v4[kFinBatch][4];
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) v4[i] = __ldcg(src + i);
+                                for (int cc = 0; cc < kFinBatch; ++cc) {
+                                    const long long ci = c0 + cc;
+                                    if (ci <= ghi) {
+                                        const int sl = ci == glo ? glo_slot : 0;
+                                        const float4* src = reinterpret_cast<const float4*>(
+                                            rowp + (ci * 2 + sl) * (long long)kVSlotFloats + m0);
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    sum[4 * i] += v4[i].x;
-                                    sum[4 * i + 1] += v4[i].y;
-                                    sum[4 * i + 2] += v4[i].z;
-                                    sum[4 * i + 3] += v4[i].w;
+                                        for (int i = 0; i < 4; ++i) v4[cc][i] = __ldcg(src + i);
+                                    }
+                                }
+#pragma unroll
+                                for (int cc = 0; cc < kFinBatch; ++cc) {
+                                    if (c0 + cc <= ghi) {
+#pragma unroll
+                                        for (int i = 0; i < 4; ++i) {
+                                            sum[4 * i] += v4[cc][i].x;
+                                            sum[4 * i + 1] += v4[cc][i].y;
+                                            sum[4 * i + 2] += v4[cc][i].z;
+                                            sum[4 * i + 3] += v4[cc][i].w;
+                                        }
+                                    }
                                 }
                             }
                             if (row_g < p.N) {
@@ -471,63 +574,58 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
                     }
                 }
             }
-            // the next chunk's buffers: wait until the MMAs that last read them are done,
-            // then store its X (rows past M, columns past K: zero)
-            if (j + 1 < n) {
-                const int b1 = (j + 1) % kVBufs;  // last used by chunk j + 1 - kVBufs
-                if (j + 1 >= kVBufs &&
-                    !vwait(bars + 8 * (kBarEmpty + b1), (uint32_t)((((j + 1) / kVBufs) - 1) & 1), abort)) {
-                    if (lane == 0 && !*abort) vabort(abort, 1u);
-                    pend_lo = j + 1;
-                    pend_hi = (j + 1 + kVStages < n) ? j + 1 + kVStages : n;
-                    break;
-                }
-                // the MMAs that read this buffer's A (tensor memory) are done: later stores follow them
-                tc_fence_after();
-                store_x(b1, xr);
-            }
-            if (++c == (int)KC) {
-                c = 0;
-                ++group;
+            group = group1;
+            pr = pr1;
+            nw = nw1;
+#pragma unroll
+            for (int h = 0; h < kVUPW; ++h) {
+                sw[h] = sw1[h];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q[h][i] = q1[h][i];
             }
         }
-        // after an abort: wait (bounded) for this warp's copies still in flight
-        for (int s = pend_lo; s < pend_hi; ++s)
-            if (tile_ok(s)) warp_wait(rbar + 8 * (s % kVStages), (uint32_t)((s / kVStages) & 1));
-    } else {
+        if (!ok) {
+            if (lane == 0 && !*abort) vabort(abort, 1u);
+            // wait (bounded) for this warp's copies still in flight
+            for (int s = waited; s < issued; ++s)
+                if (stage_units(u0 + s) > 0) warp_wait(rbar + 8 * (s % kVStages), (uint32_t)((s / kVStages) & 1));
+        }
+    } else if (warp < kVXWarp) {
+        // The MMAs of tile tt = warp - kVMmaWarp, issued by one thread: two issuers on
+        // two sub-partitions halve the issue work that competes with the dequantisation
+        // warps there.  Each tile has its own accumulator, so the two streams of MMAs
+        // need no order between them.
         if (lane == 0) {
-            int seg = 0;
+            const int tt = warp - kVMmaWarp;
+            const uint32_t d = tmem + (uint32_t)(tt * p.NL);
+            const uint32_t xoff = (uint32_t)(p.NL * 128) >> 4;  // second chunk of a buffer, in 16-byte steps
             bool any = false;
-            int c = (int)(u0 % KC) - 1;
+            int pr = pr0;
             for (int j = 0; j < n; ++j) {
-                if (++c == (int)KC) c = 0;
                 const int b = j % kVBufs;
-                const bool first = j == 0 || c == 0;
+                const int nch = 2 * pr + 1 < KC ? 2 : 1;
+                const bool first = j == 0 || pr == 0;
                 if (!vwait1(bars + 8 * (kBarFull + b), (uint32_t)((j / kVBufs) & 1), abort)) {
                     if (!*abort) vabort(abort, 2u);
                     break;
                 }
-                // the previous group's accumulators have been read back before they are overwritten
-                if (first && seg > 0 && !vwait1(bars + 8 * kBarAccFree, (uint32_t)((seg - 1) & 1), abort)) {
-                    if (!*abort) vabort(abort, 2u);
-                    break;
-                }
                 tc_fence_after();
-                const uint32_t xs = base + kOffX + b * kXBytes;
+                // X chunk h of buffer b, MMA step s at 256 s bytes (16 s in the
+                // descriptor's address field); A of this tile at column 32 h + 8 s
+                const uint64_t xd = kmajor_desc(base + kOffX + b * kXBufBytes);
+                const uint32_t a0 = tmem + (uint32_t)(kATmemCol + (b * kVTiles + tt) * kATmemTileCols);
+                tc_mma_ts(d, a0, xd, p.idesc, first ? 0u : 1u);
 #pragma unroll
-                for (int tt = 0; tt < kVTiles; ++tt) {
-                    const uint32_t at = tmem + (uint32_t)(kATmemCol + (b * kVTiles + tt) * kATmemTileCols);
+                for (int kk = 1; kk < 4; ++kk) tc_mma_ts(d, a0 + (uint32_t)(8 * kk), xd + (uint64_t)(16 * kk), p.idesc, 1u);
+                if (nch == 2) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_ts(tmem + (uint32_t)(tt * p.NL), at + (uint32_t)(8 * kk), kmajor_desc(xs + 256 * kk),
-                                  p.idesc, (first && kk == 0) ? 0u : 1u);
+                        tc_mma_ts(d, a0 + (uint32_t)(32 + 8 * kk), xd + (uint64_t)(xoff + 16 * kk), p.idesc, 1u);
                 }
                 any = true;
-                tc_commit(bars + 8 * (kBarEmpty + b));
-                if (c == (int)KC - 1 || j == n - 1) {
-                    tc_commit(bars + 8 * kBarAcc);
-                    ++seg;
-                }
+                tc_commit(bars + 8 * (kBarFree + b));
+                if (pr == KP - 1 || j == n - 1) tc_commit(bars + 8 * kBarAcc);
+                if (++pr == KP) pr = 0;
             }
             // every MMA finished before the tensor memory is released
             if (any) {
@@ -537,10 +635,40 @@ __global__ void __launch_bounds__(kVThreads, kVCtasPerSM) verify_kernel(const VP
             }
         }
         __syncwarp();
+    } else if (warp == kVXWarp) {
+        if (lane == 0) {
+            // Xp is written by the preceding kernel
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            const uint64_t pol = evict_last_policy();
+            int pr = pr0, issued = 0;
+            for (int j = 0; j < n; ++j) {
+                const int b = j % kVBufs;
+                // buffer b was last read by the MMAs of hand-off j - kVBufs
+                if (j >= kVBufs && !vwait1(bars + 8 * (kBarFree + b), (uint32_t)(((j / kVBufs) - 1) & 1), abort)) {
+                    if (!*abort) vabort(abort, 2u);
+                    break;
+                }
+                const int nch = 2 * pr + 1 < KC ? 2 : 1;
+                const uint32_t bytes = (uint32_t)(nch * p.NL * 128);
+                const uint32_t bar = bars + 8 * (kBarFull + b);
+                mbar_expect_tx(bar, bytes);  // also this thread's arrival on full[b]
+                bulk_load(base + kOffX + b * kXBufBytes, p.Xp + (long long)(2 * pr) * p.NL * 128, bytes, bar, pol);
+                issued = j + 1;
+                if (++pr == KP) pr = 0;
+            }
+            // After an abort the last copies may still be in flight: wait (bounded) for
+            // their phases, which complete once they land unless a warp's arrival is
+            // missing too, in which case the wait runs out well after they landed.
+            if (*abort)
+                for (int j = issued > kVBufs ? issued - kVBufs : 0; j < issued; ++j)
+                    for (uint32_t it = 0; it < kWaitLimit; ++it)
+                        if (mbar_try_wait(bars + 8 * (kBarFull + j % kVBufs), (uint32_t)((j / kVBufs) & 1))) break;
+        }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kVWarps) {
+    if (warp == kVMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols)
                      : "memory");
@@ -557,31 +685,49 @@ struct VerifyState {
     int max_ctas = 0;
     float* part = nullptr;
     unsigned* counters = nullptr;
+    uint8_t* xp = nullptr;  // X in the MMA's order, rewritten by every call
+    size_t xp_bytes = 0;
 };
 std::mutex g_vmu;
 VerifyState g_vstate[64];
 
-int verify_state(cudaStream_t stream, VerifyState** out)
+constexpr size_t kXpInitialBytes = (size_t)kVMaxNL * 128 * 1024;  // K up to 65,536 at nl = 64: 8 MB
+
+int verify_state(cudaStream_t stream, size_t xp_need, VerifyState** out)
 {
     int dev = 0;
     NVFP4_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return NVFP4_ERR_ARG;
     std::lock_guard<std::mutex> lock(g_vmu);
     VerifyState& s = g_vstate[dev];
-    if (s.device == dev) {
+    if (s.device == dev && s.xp_bytes >= xp_need) {
         *out = &s;
         return NVFP4_OK;
     }
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     NVFP4_CUDA_TRY(cudaStreamIsCapturing(stream, &cs));
     if (cs != cudaStreamCaptureStatusNone) return NVFP4_ERR_CAPTURE;
+    if (s.device == dev) {
+        // a longer K than before: a larger X buffer, once nothing uses the old one
+        NVFP4_CUDA_TRY(cudaDeviceSynchronize());
+        NVFP4_CUDA_TRY(cudaFree(s.xp));
+        s.xp = nullptr;
+        s.xp_bytes = 0;
+        NVFP4_CUDA_TRY(cudaMalloc(&s.xp, xp_need));
+        s.xp_bytes = xp_need;
+        *out = &s;
+        return NVFP4_OK;
+    }
     int sms = 0;
     NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int max_ctas = kVCtasPerSM * sms;
+    const size_t xp_bytes = xp_need > kXpInitialBytes ? xp_need : kXpInitialBytes;
     float* part = nullptr;
     unsigned* counters = nullptr;
+    uint8_t* xp = nullptr;
     NVFP4_CUDA_TRY(cudaMalloc(&part, (size_t)max_ctas * 2 * kVSlotFloats * sizeof(float)));
     cudaError_t e = cudaMalloc(&counters, (size_t)kVMaxGroups * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMalloc(&xp, xp_bytes);
     if (e == cudaSuccess) e = cudaMemset(counters, 0, (size_t)kVMaxGroups * sizeof(unsigned));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kVSmemBytes);
@@ -589,12 +735,15 @@ int verify_state(cudaStream_t stream, VerifyState** out)
     if (e != cudaSuccess) {
         cudaFree(part);
         if (counters) cudaFree(counters);
+        if (xp) cudaFree(xp);
         return fail_cuda(e);
     }
     s.sm_count = sms;
     s.max_ctas = max_ctas;
     s.part = part;
     s.counters = counters;
+    s.xp = xp;
+    s.xp_bytes = xp_bytes;
     s.device = dev;
     *out = &s;
     return NVFP4_OK;
@@ -608,18 +757,19 @@ int verify_geometry(int M, int64_t N, int64_t K, int sm_count, VerifyGeometry* g
     int st = check_shape(N, K);
     if (st != NVFP4_OK) return st;
     g->n_tiles32 = (N + kTileN - 1) / kTileN;
-    g->n_groups = (g->n_tiles32 + kVWarps - 1) / kVWarps;  // groups of kVWarps 32-row tiles
+    g->n_groups = (g->n_tiles32 + kVSlices - 1) / kVSlices;  // groups of kVSlices 32-row tiles
     if (g->n_groups > kVMaxGroups) return NVFP4_ERR_SHAPE;
     g->k_chunks = (K + kChunkK - 1) / kChunkK;
-    g->units = g->n_groups * g->k_chunks;
-    // one CTA per SM, but no more than kVMaxSplit CTAs per tile group on average: a group
+    g->k_pairs = (g->k_chunks + kVPair - 1) / kVPair;
+    g->units = g->n_groups * g->k_pairs;
+    // one CTA per SM, but no more than kVMaxSplit CTAs per group on average: a group
     // split between more CTAs costs more in partial sums than the extra SMs stream
     long long ctas = (long long)kVCtasPerSM * sm_count;
     if (ctas > g->n_groups * kVMaxSplit) ctas = g->n_groups * kVMaxSplit;
     if (ctas > g->units) ctas = g->units;
     g->ctas = ctas;
     g->nl = (M + 15) / 16 * 16;
-    g->tmem_cols = kVTmemCols;  // accumulators (4 x nl <= 256 columns) and the double-buffered A operand
+    g->tmem_cols = kVTmemCols;  // accumulators (2 x nl <= 128 columns) and the triple-buffered A operand
     return NVFP4_OK;
 }
 
@@ -631,8 +781,9 @@ int launch_verify(const void* X, int M, const uint8_t* wq, const uint8_t* ws, fl
     int st = check_shape(N, K);
     if (st != NVFP4_OK) return st;
     if (!aligned16(X) || !aligned16(wq) || !aligned16(ws) || ((uintptr_t)Y & 3) != 0) return NVFP4_ERR_ALIGN;
+    const long long pieces = (K + kChunkK - 1) / kChunkK * ((M + 15) / 16 * 16) * 8;  // 16-byte pieces of X
     VerifyState* vs = nullptr;
-    st = verify_state(stream, &vs);
+    st = verify_state(stream, (size_t)pieces * 16, &vs);
     if (st != NVFP4_OK) return st;
     VerifyGeometry geo;
     st = verify_geometry(M, N, K, vs->sm_count, &geo);
@@ -640,7 +791,7 @@ int launch_verify(const void* X, int M, const uint8_t* wq, const uint8_t* ws, fl
     VParams p;
     p.wq = wq;
     p.ws = ws;
-    p.X = static_cast<const uint16_t*>(X);
+    p.Xp = vs->xp;
     p.Y = Y;
     p.part = vs->part;
     p.counters = vs->counters;
@@ -649,24 +800,29 @@ int launch_verify(const void* X, int M, const uint8_t* wq, const uint8_t* ws, fl
     p.NL = geo.nl;
     p.tmem_cols = geo.tmem_cols;
     p.N = N;
-    p.K = K;
     p.KC = (int)geo.k_chunks;
+    p.KP = (int)geo.k_pairs;
     p.n_tiles32 = (int)geo.n_tiles32;
     p.n_groups = (int)geo.n_groups;
     p.units = geo.units;
     p.ctas = geo.ctas;
     // kind::f16 instruction: F32 accumulator, BF16 A and B, both K-major, N = nl, M = 128
     p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(geo.nl >> 3) << 17) | ((uint32_t)(kVTileRows >> 4) << 24);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)geo.ctas);
-    cfg.blockDim = dim3(kVThreads);
-    cfg.dynamicSmemBytes = kVSmemBytes;
-    cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((pieces + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, verify_xprep_kernel, static_cast<const uint16_t*>(X), vs->xp, M,
+                                      geo.nl, (long long)K, pieces));
+    cfg.gridDim = dim3((unsigned)geo.ctas);
+    cfg.blockDim = dim3(kVThreads);
+    cfg.dynamicSmemBytes = kVSmemBytes;
     NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, verify_kernel, p));
     return NVFP4_OK;
 }

@@ -198,13 +198,14 @@ def test_host_layout_model_every_code_with_every_scale(lib):
                                  (151936, 5120), (1000, 1040)])
 def test_verify_geometry(lib, M, N, K):
     """Work split of the verify-width kernel: every CTA owns a non-empty range
-    of (512-row tile group, chunk) units, one CTA per SM at most, no more than
-    4 CTAs per group on average, and the MMA's N is M rounded up to 16."""
+    of (256-row group, pair of 64-column chunks) units, one CTA per SM at
+    most, no more than 8 CTAs per group on average, and the MMA's N is M
+    rounded up to 16."""
     st, ctas, units, nl = abi.nvfp4_verify_geometry(M, N, K, 148)
     assert st == abi.NVFP4_OK
-    groups = -(-(-(-N // 32)) // 16)
-    assert units == groups * -(-K // 64)
-    assert 1 <= ctas <= min(148, units, 4 * groups)
+    groups = -(-(-(-N // 32)) // 8)
+    assert units == groups * -(-(-(-K // 64)) // 2)
+    assert 1 <= ctas <= min(148, units, 8 * groups)
     assert nl % 16 == 0 and M <= nl < M + 16
     assert all(units * (i + 1) // ctas > units * i // ctas for i in range(ctas))
 
