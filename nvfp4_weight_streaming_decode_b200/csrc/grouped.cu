@@ -14,8 +14,8 @@
 // deterministic way -- valid routes sorted by (expert, route position), runs
 // of one expert cut into groups of at most 8 rows (the MMA's lane side) --
 // and the selected groups' units are concatenated into one virtual matrix
-// that the warps split evenly (stream-K), each block of rows coming from its
-// own expert's planes and its own X rows.  Split-K partial sums are combined
+// that the warps split evenly (stream-K, at least one 4-unit stage per warp),
+// each block of rows coming from its own expert's planes and its own X rows.  Split-K partial sums are combined
 // by the last contributor in warp order, as in the decode GEMM.  Routes whose
 // expert id is outside 0..E-1, or whose planes are not 16-byte aligned, give
 // zero rows and set a device status bit.  Every wait is bounded; no CTA waits
@@ -42,6 +42,11 @@ constexpr int kGStages = 3;     // per-warp ring depth
 constexpr int kGUPS = 4;        // units per stage (a stage crossing to the next expert takes one copy per part)
 constexpr int kGStage = kGUPS * kUnitBytes;
 constexpr int kGSlot = 256;     // a partial: 32 lanes x 8 floats
+// Units per warp at least: a small call (M = 1: ten experts) runs on fewer
+// warps, each with one full stage in flight and fewer split-K partials per
+// tile (measured at M = 1, T = 10 on 768 x 2,048 experts: 1 unit 11.0 us,
+// 2-3 units 10.8-10.9, 4 units 9.4, 5-6 units 11.0-11.3, 8 units 11.3).
+constexpr int kGMinUnits = kGUPS;
 constexpr int kGMaxTiles = 4096;  // 32-row tiles per expert (N <= 131,072)
 
 struct GParams {
@@ -100,12 +105,15 @@ struct GroupTable {
     int g_rows[NVFP4_GROUPED_MAX_ROUTES];    // per group: rows, 1..8
     int start[NVFP4_GROUPED_MAX_ROUTES];     // per sorted position: 1 if it starts a group
     int exp[NVFP4_GROUPED_MAX_ROUTES];       // per route: its expert, or -1 (no expert / invalid)
+    // per route: its expert's planes and scale, read once while grouping, so that
+    // the copies and the epilogue need no further read of the expert table
+    const uint8_t* r_wq[NVFP4_GROUPED_MAX_ROUTES];
+    const uint8_t* r_ws[NVFP4_GROUPED_MAX_ROUTES];
+    float r_gs[NVFP4_GROUPED_MAX_ROUTES];
 };
 
-__device__ __forceinline__ bool expert_ok(const GParams& p, int e)
+__device__ __forceinline__ bool expert_ok(const nvfp4_expert& ex)
 {
-    if (e < 0 || e >= p.E) return false;
-    const nvfp4_expert ex = p.experts[e];
     return ex.wq && ex.ws && (((uintptr_t)ex.wq | (uintptr_t)ex.ws) & 15u) == 0;
 }
 
@@ -118,7 +126,15 @@ __device__ void build_groups(const GParams& p, GroupTable& gt)
     const int tid = threadIdx.x;
     if (tid < R) {
         const int e = p.route[tid];
-        gt.exp[tid] = expert_ok(p, e) ? e : -1;
+        bool ok = e >= 0 && e < p.E;
+        if (ok) {
+            const nvfp4_expert ex = p.experts[e];
+            ok = expert_ok(ex);
+            gt.r_wq[tid] = ex.wq;
+            gt.r_ws[tid] = ex.ws;
+            gt.r_gs[tid] = ex.gscale;
+        }
+        gt.exp[tid] = ok ? e : -1;
     }
     // every thread sees the count of valid routes
     const int nv = __syncthreads_count(tid < R && gt.exp[tid] >= 0);
@@ -201,8 +217,11 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
     }
 
     const long long U = gt.n_groups * p.UE;
+    // at least kGMinUnits units per warp: for small calls fewer warps, each with
+    // more copies in flight, and fewer split-K partials per tile
     const long long TWmax = (long long)gridDim.x * kGWarps;
-    const long long TW = TWmax < U ? TWmax : U;
+    const long long TWu = (U + kGMinUnits - 1) / kGMinUnits;
+    const long long TW = TWmax < TWu ? TWmax : TWu;
     if (gw >= TW) return;  // (no CTA-wide barrier follows)
     const long long KC = p.KC, UE = p.UE;
     const long long u0 = g_range_begin(U, TW, gw), u1 = g_range_begin(U, TW, gw + 1);
@@ -224,9 +243,9 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
             // the longest run of this stage's units within one expert
             const long long left = UE - iul;
             const int part = (long long)(cnt - v) < left ? cnt - v : (int)left;
-            const nvfp4_expert ex = p.experts[gt.g_expert[ig]];
-            bulk_load(dst + v * kUnitQ, ex.wq + iul * kUnitQ, part * kUnitQ, bar, pol);
-            bulk_load(dst + kGUPS * kUnitQ + v * kUnitS, ex.ws + iul * kUnitS, part * kUnitS, bar, pol);
+            const int r0 = gt.sorted[gt.g_first[ig]];  // a route of this group: its expert's planes
+            bulk_load(dst + v * kUnitQ, gt.r_wq[r0] + iul * kUnitQ, part * kUnitQ, bar, pol);
+            bulk_load(dst + kGUPS * kUnitQ + v * kUnitS, gt.r_ws[r0] + iul * kUnitS, part * kUnitS, bar, pol);
             v += part;
             iul += part;
             if (iul == UE) {
@@ -252,7 +271,7 @@ __global__ void __launch_bounds__(kGWarps * 32, 1) grouped_kernel(const GParams 
     auto set_group = [&]() {
         rows = gt.g_rows[grp];
         first = gt.g_first[grp];
-        gscale = p.experts[gt.g_expert[grp]].gscale;
+        gscale = gt.r_gs[gt.sorted[first]];
         // past the group's rows a lane loads its first row, which feeds only dropped output columns
         const int pos = gt.sorted[first + (g8 < rows ? g8 : 0)];
         xrow = p.X + (long long)(p.x_per_route ? pos : pos / p.T) * p.K;
