@@ -59,7 +59,13 @@ __device__ unsigned int g_verify_status;
 
 namespace {
 
-constexpr int kVTiles = 2;                       // 128-row MMA tiles per group (256 rows)
+// 128-row MMA tiles per group.  One tile runs two CTAs per SM (each with half
+// the tensor memory): faster on the head at M = 64 (203 against 210 us), slower
+// on the shapes with few groups (down at M = 40: 62 against 51 us).
+#ifndef NVFP4_VTILES
+#define NVFP4_VTILES 2
+#endif
+constexpr int kVTiles = NVFP4_VTILES;
 constexpr int kVSlices = 4 * kVTiles;            // 32-row slices per group
 constexpr int kVPair = 2;                        // 64-column chunks per hand-off
 #ifndef NVFP4_VSPLIT
@@ -70,11 +76,11 @@ constexpr int kVWarps = kVSlices * kVSplit;
 constexpr int kVUPW = kVPair / kVSplit;          // units per warp and hand-off
 static_assert(kVPair % kVSplit == 0, "the chunks of a hand-off divide among a slice's warps");
 constexpr int kVBufs = 3;                        // hand-offs in flight: A buffers (tensor memory), X buffers (shared)
-constexpr int kVStages = 7;                      // per-warp ring depth, one hand-off per stage
+constexpr int kVStages = kVTiles == 1 ? 6 : 7;   // per-warp ring depth, one hand-off per stage
 constexpr int kVMmaWarp = kVWarps;               // one thread per tile issues its MMAs (warps kVWarps..)
 constexpr int kVXWarp = kVWarps + kVTiles;       // one thread stages X
 constexpr int kVThreads = (kVXWarp + 1) * 32;
-constexpr int kVCtasPerSM = 1;                   // one CTA per SM: it holds all 512 tensor-memory columns
+constexpr int kVCtasPerSM = kVTiles == 1 ? 2 : 1;  // CTAs per SM, sharing the 512 tensor-memory columns
 constexpr int kVTileRows = 128;                  // MMA M
 constexpr int kVMaxNL = 64;                      // MMA N at most (M rows of X, padded to 16)
 constexpr int kVGroupRows = kVTiles * kVTileRows;        // 256
@@ -84,7 +90,7 @@ constexpr int kXBufBytes = kVPair * kXChunkBytes;        // 16 KB
 // Tensor memory (512 columns): accumulators in columns [0, kVTiles * nl)
 // (nl <= 64); the bf16 A operand from column 128: per buffer and tile, 128
 // lanes x 64 columns (a hand-off's 128 values per row, two per column).
-constexpr int kVTmemCols = 512;
+constexpr int kVTmemCols = 512 / kVCtasPerSM;
 constexpr int kATmemCol = kVTiles * kVMaxNL;             // 128
 constexpr int kATmemTileCols = kVPair * kChunkK / 2;     // 64
 static_assert(kATmemCol + kVBufs * kVTiles * kATmemTileCols <= kVTmemCols, "tensor memory holds A and D");
@@ -104,7 +110,7 @@ constexpr int kBarRing = 0, kBarFull = kVWarps * kVStages, kBarFree = kBarFull +
               kBarPart = kBarAcc + 1, kBarLast = kBarPart + 1, kBarFin = kBarLast + 1, kNumBars = kBarFin + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;                  // tmem base, abort, last, pad
 constexpr int kVSmemBytes = kOffMisc + 16;
-static_assert(kVSmemBytes <= 227 * 1024, "shared memory per CTA");
+static_assert(kVSmemBytes * kVCtasPerSM <= 226 * 1024, "shared memory per SM");
 
 struct VParams {
     const uint8_t* wq;
