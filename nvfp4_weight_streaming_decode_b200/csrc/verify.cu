@@ -59,13 +59,10 @@ __device__ unsigned int g_verify_status;
 
 namespace {
 
-// 128-row MMA tiles per group.  One tile runs two CTAs per SM (each with half
-// the tensor memory): faster on the head at M = 64 (203 against 210 us), slower
-// on the shapes with few groups (down at M = 40: 62 against 51 us).
-#ifndef NVFP4_VTILES
-#define NVFP4_VTILES 2
-#endif
-constexpr int kVTiles = NVFP4_VTILES;
+// 128-row MMA tiles per group.  (One tile with two CTAs per SM, each with half
+// the tensor memory, measured faster on the head at M = 64 -- 203 against
+// 210 us -- but slower where groups are few: down at M = 40 62 against 51 us.)
+constexpr int kVTiles = 2;
 constexpr int kVSlices = 4 * kVTiles;            // 32-row slices per group
 constexpr int kVPair = 2;                        // 64-column chunks per hand-off
 #ifndef NVFP4_VSPLIT
