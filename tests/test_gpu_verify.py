@@ -112,3 +112,16 @@ def test_wide_width_is_deterministic_and_matches_per_block_rows(dev):
     Yr, A = oracle.gemm(X, q, s, synth.GSCALE)
     assert_gemm_close(Y1[:8].cpu().numpy(), Yr[:8], A[:8], "lanes 0..7")
     assert_gemm_close(Y1[8:].cpu().numpy(), Yr[8:], A[8:], "lanes 8..12")
+
+
+def test_verify_long_k_grows_the_x_buffer(dev):
+    """K past 65,536 at a verify width: the first such call grows the buffer
+    that holds X in the MMA's order (outside any capture), and both that call
+    and a shorter one after it agree with the oracle."""
+    N = 64
+    for K in (65536 + 1024, 2048):
+        q, s = synth.matrix(55, K, N, K)
+        X = synth.activations(synth.rng(55, K), 40, K)
+        Y = gemm_case(dev, q, s, X)
+        Yr, A = oracle.gemm(X, q, s, synth.GSCALE)
+        assert_gemm_close(Y, Yr, A, f"M=40 N={N} K={K}")
